@@ -1,0 +1,440 @@
+"""Benchmark of the sparse absorbed MLA decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one call of the whole decode path (absorb, sparse attend, combine +
+value-up) over one batch of B rows.  The default workload is the B=64,
+32K-context, top-2048 configuration.  Inputs are synthetic (seeded), generated
+on the host in bf16 and kept resident in HBM; NSETS independent input sets
+(queries, index sets, end positions and a separate copy of wkv_b each) rotate
+between steps, so a step never finds the previous step's bytes in L2.
+
+Prints one JSON line (rank 0).  Under torchrun every rank runs its own batch
+(weak scaling, no collective on the path); the step time is the maximum over
+ranks.  ``--impl reference`` times the fp64 CPU oracle on a bounded sample of
+the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from sparse_latent_attention_absorb_b200 import workloads as wl  # noqa: E402
+
+DEFAULT_WORKLOAD = "b64_ctx1k-32k_top2048"
+NSETS = 4
+METRIC = "sparse MLA decode queries/s"
+UNIT = "queries/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def algorithmic(B, K, sum_k):
+    """Bytes and FLOPs the method must move / compute for one call (no dense
+    mask, no split partials): wkv_b once, the queries, the gathered latent +
+    rotary rows of every selected position, the indices, end_pos and out."""
+    bytes_ = (128 * 256 * 512 * 2 + B * 128 * (128 + 64) * 2 + 1152 * sum_k + 4 * B * K + 4 * B + B * 128 * 128 * 2)
+    flops = 2 * 128 * 128 * 512 * 2 * B + 2 * 128 * (576 + 512) * sum_k
+    return bytes_, flops
+
+
+def attend_bytes(B, K, sum_k):
+    """Algorithmic bytes of the sparse-attend kernel alone: the gathered rows
+    (1152 B per selected position), the indices and end_pos."""
+    return 1152 * sum_k + 4 * B * K + 4 * B
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for f in ("kernels.cuh", "ptx.cuh", "mla_sparse_decode.cu"):
+        with open(os.path.join(ROOT, "sparse_latent_attention_absorb_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    """DRAM bytes per launch of the sparse-attend kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        e = t.get(workload)
+        if e and e.get("source_hash") == source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def make_sets(w, device):
+    """NSETS input sets on the device: the caches are shared (model state),
+    everything else is drawn per set."""
+    base = wl.generate(w)
+    caches = {k: base[k].to(device) for k in ("kv_cache", "pe_cache")}
+    sets = []
+    for i in range(NSETS):
+        d = base if i == 0 else wl.generate(w, seed_offset=i, caches=False)
+        s = {k: d[k].to(device) for k in ("q_nope", "q_pe", "end_pos", "topk_idx", "wkv_b")}
+        s.update(caches)
+        s["scale"] = d["scale"]
+        s["sum_k"] = wl.selected_count(d["end_pos"], d["topk_idx"])
+        s["host"] = d
+        sets.append(s)
+    return sets, base
+
+
+def gpu_arm(args, rank, world, device):
+    import ctypes
+
+    import sparse_latent_attention_absorb_b200 as pkg
+    from sparse_latent_attention_absorb_b200 import binding
+
+    lib = pkg.load_library()
+    w = wl.ALL_WORKLOADS[args.workload]
+    sets, base = make_sets(w, device)
+    B, K, S_max = w.B, w.K, w.S_max
+    n_split = pkg.num_splits(B, K)
+    ws = torch.empty(pkg.workspace_size(B, K, S_max), dtype=torch.uint8, device=device)
+    outs = [torch.empty((B, 128, 128), dtype=torch.bfloat16, device=device) for _ in sets]
+    stream = torch.cuda.Stream(device=device)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+
+    def call(i, st):
+        s = sets[i]
+        rc = lib.mla_sparse_decode(P(s["q_nope"]), P(s["q_pe"]), P(s["kv_cache"]), P(s["pe_cache"]), P(s["end_pos"]),
+                                   P(s["topk_idx"]), P(s["wkv_b"]), ctypes.c_float(s["scale"]), P(outs[i]), B, K,
+                                   S_max, P(ws), ws.numel(), None, None, ctypes.c_void_p(st.cuda_stream))
+        if rc != 0:
+            raise binding.MLAError(rc, "mla_sparse_decode")
+
+    # one CUDA graph per input set: a replay is exactly one decode call
+    with torch.cuda.stream(stream):
+        for i in range(len(sets)):
+            call(i, stream)
+    stream.synchronize()
+    graphs = []
+    for i in range(len(sets)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            call(i, torch.cuda.current_stream())
+        graphs.append(g)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # ---- timed region: K decode steps
+    with torch.cuda.stream(stream):
+        for it in range(args.warmup):
+            graphs[it % NSETS].replay()
+    stream.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device() if device.index is None else device.index) as clocks:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for it in range(args.steps):
+                graphs[it % NSETS].replay()
+            ev1.record(stream)
+        stream.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    value = B * world * args.steps / (elapsed_ms / 1e3)
+    launches = 3 * args.steps
+
+    # ---- per-kernel live timing (same stream, back-to-back launches, sets rotate)
+    q_lat = [torch.empty((B, 128, 512), dtype=torch.bfloat16, device=device) for _ in sets]
+    o_part = torch.empty((B, n_split, 128, 512), dtype=torch.float32, device=device)
+    lse_part = torch.empty((B, n_split, 128), dtype=torch.float32, device=device)
+    sv = ctypes.c_void_p(stream.cuda_stream)
+
+    def k_absorb(i):
+        return lib.mla_absorb_q(P(sets[i]["q_nope"]), P(sets[i]["wkv_b"]), P(q_lat[i]), B, sv)
+
+    def k_attend(i):
+        s = sets[i]
+        return lib.mla_sparse_attend(P(q_lat[i]), P(s["q_pe"]), P(s["kv_cache"]), P(s["pe_cache"]), P(s["end_pos"]),
+                                     P(s["topk_idx"]), ctypes.c_float(s["scale"]), P(o_part), P(lse_part), B, K,
+                                     S_max, n_split, None, sv)
+
+    def k_combine(i):
+        return lib.mla_combine_value_up(P(o_part), P(lse_part), P(sets[i]["wkv_b"]), P(outs[i]), None, B, n_split, sv)
+
+    def time_kernel(fn, reps):
+        with torch.cuda.stream(stream):
+            for r in range(4):
+                assert fn(r % NSETS) == 0
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for r in range(reps):
+                fn(r % NSETS)
+            e1.record(stream)
+        stream.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    with torch.cuda.stream(stream):
+        for i in range(NSETS):
+            k_absorb(i)
+    stream.synchronize()
+    reps = max(20, args.steps)
+    t_absorb = time_kernel(k_absorb, reps)
+    t_attend = time_kernel(k_attend, reps)
+    t_combine = time_kernel(k_combine, reps)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if rank == 0 or world > 1:
+        import sparse_latent_attention_absorb_b200 as api
+        hsets = []
+        for s in sets:
+            h = s["host"]
+            hsets.append({k: h[k].pin_memory() for k in ("q_nope", "q_pe", "end_pos", "topk_idx")})
+        dev_in = {k: torch.empty_like(sets[0][k]) for k in ("q_nope", "q_pe", "end_pos", "topk_idx")}
+        out_host = torch.empty((B, 128, 128), dtype=torch.bfloat16).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in hsets[0].values())
+        d2h = out_host.numel() * out_host.element_size()
+
+        def e2e_step(i):
+            for k, v in hsets[i].items():
+                dev_in[k].copy_(v, non_blocking=True)
+            api.mla_sparse_decode(dev_in["q_nope"], dev_in["q_pe"], sets[i]["kv_cache"], sets[i]["pe_cache"],
+                                  dev_in["end_pos"], dev_in["topk_idx"], sets[i]["wkv_b"], sets[i]["scale"],
+                                  out=outs[i], workspace=ws)
+            out_host.copy_(outs[i], non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for it in range(max(3, args.warmup)):
+                e2e_step(it % NSETS)
+        stream.synchronize()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            f0.record(stream)
+            for it in range(args.steps):
+                e2e_step(it % NSETS)
+            f1.record(stream)
+        stream.synchronize()
+        e_ms = f0.elapsed_time(f1)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=device)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": B * world * args.steps / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+
+    # ---- roofline of the dominant kernel and of the whole call
+    hbm, tf, tf_sus, kind = peaks()
+    sum_k = statistics.mean(s["sum_k"] for s in sets)
+    a_bytes = attend_bytes(B, K, sum_k)
+    achieved = a_bytes / (t_attend * 1e-3) / 1e9
+    traffic = ncu_traffic(args.workload)
+    call_bytes, call_flops = algorithmic(B, K, sum_k)
+    t_hbm = call_bytes / (hbm * 1e9)
+    t_tc = call_flops / (tf * 1e12)
+    roof_ms = max(t_hbm, t_tc) * 1e3
+
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "B": B, "heads": 128, "S_max": S_max, "K": K,
+                   "end_pos": list(w.end_pos), "index": w.index, "sum_k_mean": sum_k, "splits": n_split,
+                   "parallelism": f"replicas x{world} (batch rows)",
+                   "l2": f"{NSETS} rotating input sets (queries, indices, wkv_b copy each); per-step footprint "
+                         f"{call_bytes / 1e6:.0f} MB > 126 MB L2",
+                   "timing": "CUDA graph replay per step, CUDA events on the launching stream"},
+        "roofline": {"bound": "hbm", "kernel": "sparse_attend_kernel", "achieved": achieved, "peak": hbm,
+                     "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
+                     "peak_source": f"{kind} hbm_gbs", "alg_bytes_per_launch": a_bytes,
+                     "ms_per_launch": t_attend},
+        "call_roofline": {"alg_bytes": call_bytes, "alg_flops": call_flops, "t_hbm_ms": t_hbm * 1e3,
+                          "t_tensor_ms": t_tc * 1e3, "roofline_ms": roof_ms, "frac": roof_ms / ms_per_step,
+                          "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                          "peaks": {"hbm_gbs": hbm, "bf16_tflops": tf, "source": kind}},
+        "kernels_ms": {"absorb": t_absorb, "sparse_attend": t_attend, "combine_value_up": t_combine},
+        "gpu_launches": launches,
+        "e2e": e2e,
+        "clocks": clocks.summary(),
+    }
+    for g in graphs:
+        del g
+    return res, base
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(args, base, budget_s=12.0):
+    """The fp64 oracle as it stands on a bounded sample of the same workload
+    (whole batch rows, all 128 heads)."""
+    import oracle
+    w = wl.ALL_WORKLOADS[args.workload]
+    d = base
+    t0 = time.perf_counter()
+    oracle.mla_sparse_decode(d["q_nope"], d["q_pe"], d["kv_cache"], d["pe_cache"], d["end_pos"], d["topk_idx"],
+                             d["wkv_b"], d["scale"], rows=[0])
+    t1 = time.perf_counter() - t0
+    n = max(1, min(w.B, int(budget_s / max(t1, 1e-3))))
+    rows = list(range(n))
+    t0 = time.perf_counter()
+    oracle.mla_sparse_decode(d["q_nope"], d["q_pe"], d["kv_cache"], d["pe_cache"], d["end_pos"], d["topk_idx"],
+                             d["wkv_b"], d["scale"], rows=rows)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} of {w.B} batch rows (all 128 heads), one pass, {dt:.1f} s"}
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    w = wl.ALL_WORKLOADS[args.workload]
+    d = wl.generate(w)
+    times = []
+    for it in range(args.warmup + args.steps):
+        row = it % w.B
+        t0 = time.perf_counter()
+        oracle.mla_sparse_decode(d["q_nope"], d["q_pe"], d["kv_cache"], d["pe_cache"], d["end_pos"], d["topk_idx"],
+                                 d["wkv_b"], d["scale"], rows=[row])
+        if it >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = args.steps / total
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "B": w.B, "heads": 128, "S_max": w.S_max, "K": w.K},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": "each step: 1 batch row (all 128 heads) of the workload"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.ALL_WORKLOADS))
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = reference_arm(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    res, base = gpu_arm(args, rank, world, device)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(args, base["host"] if "host" in base else base)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,142 @@
+/*
+ * mla_sparse_decode.h -- C ABI of the B200 (sm_100a) sparse MLA decode library.
+ *
+ * One decode step of DeepSeek-V3.2-Exp's absorbed multi-head latent attention
+ * with the indexer's top-k mask, as the atlas pages of
+ * deepseek-ai/DeepSeek-V3.2-Exp inference/model.py (rev 87e509a2e5a1) show it:
+ *   - "Query-key similarity" (decode): MQA-decode excerpt, model.py 590-606:
+ *       absorb   q_lat = einsum("bshd,hdc->bshc", q_nope, wkv_b[:, :128])   (595)
+ *       scores   (einsum(q_lat, kv_cache) + einsum(q_pe, pe_cache)) * scale  (596-597)
+ *       mask     -inf except at topk_indices, shared by all heads          (601-602)
+ *       softmax  over key positions                                        (604)
+ *       mix      x = einsum("bsht,btc->bshc", scores, kv_cache)            (605)
+ *       value-up x = einsum("bshc,hdc->bshd", x, wkv_b[:, -128:])          (606)
+ *   - "Softmax": A = exp(S~) / sum_u exp(S~), in the scores' own type;
+ *   - "Apply value weights": O_i = O~_i W_UV,i, and A(c W_UV) = (A c) W_UV.
+ *
+ * Fixed dimensions (the pages' model): 128 heads, q_nope 128, q_pe 64,
+ * latent 512, value 128; wkv_b is [128*256, 512] = view [128 heads, 256, 512],
+ * rows 0..127 of a head are W_UK and rows 128..255 are W_UV.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE memory owned by the caller, row-major and
+ *     contiguous, 16-byte aligned.  The library allocates nothing and keeps no
+ *     state besides per-device cached launch attributes; it is reentrant.
+ *   - "bf16" pointers hold IEEE bfloat16 values (passed as void*).
+ *   - Work is enqueued on `stream` (0 = legacy default stream); no host
+ *     synchronisation happens.  An argument error is returned BEFORE anything
+ *     is launched.  A launch error returns MLA_ERR_CUDA.  Faults during
+ *     execution appear at the caller's next synchronisation; a device wait
+ *     that exceeds its time limit writes MLA_ERR_DEVICE_TIMEOUT to *d_status
+ *     (when d_status is not NULL) and the kernels return without hanging.
+ *   - Index semantics: topk_idx[b, k] selects cache position t of batch row b
+ *     when 0 <= t < min(end_pos[b], S_max); any other value (canonically -1)
+ *     is padding and is skipped.  Valid indices of one row must be distinct
+ *     (the indexer's top-k output is); a repeated index would be counted twice.
+ *     Index order is irrelevant.  A row with no valid index yields out = 0 and
+ *     lse = -inf.
+ *   - Batch row b reads cache slot b (the excerpt slices kv_cache[:bsz]).
+ */
+#ifndef MLA_SPARSE_DECODE_H
+#define MLA_SPARSE_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_HEADS 128
+#define MLA_D_NOPE 128
+#define MLA_D_ROPE 64
+#define MLA_D_LATENT 512
+#define MLA_D_V 128
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,    /* null / misaligned pointer, bad size        */
+  MLA_ERR_WORKSPACE = 2,      /* workspace missing, misaligned or too small */
+  MLA_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed       */
+  MLA_ERR_DEVICE_TIMEOUT = 4, /* written to *d_status by a timed-out wait   */
+  MLA_ERR_BAD_INDEX = 5,      /* reserved for index validation reports      */
+  MLA_ERR_UNSUPPORTED = 6     /* device is not sm_100                       */
+} mla_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* mla_status_string(int status);
+
+/* Number of key splits the decode uses for a batch of B rows with K index
+ * slots per row on the current device (a pure function of B, K and the
+ * device's SM count).  Returns 0 for invalid sizes. */
+int mla_num_splits(int B, int K);
+
+/* Bytes of scratch `mla_sparse_decode` needs for these sizes on the current
+ * device: the absorbed queries (bf16 [B,128,512]) and the per-split partial
+ * outputs (f32 [B,splits,128,512] plus f32 [B,splits,128]).  Returns 0 for
+ * invalid sizes. */
+size_t mla_sparse_decode_workspace_size(int B, int K, int S_max);
+
+/*
+ * The whole decode step (steps absorb .. value-up above).
+ *   q_nope   bf16 [B,128,128]   non-rotary queries
+ *   q_pe     bf16 [B,128,64]    rotary queries, already rotated
+ *   kv_cache bf16 [B,S_max,512] normalised latent cache c^KV
+ *   pe_cache bf16 [B,S_max,64]  rotated shared rotary key k^R
+ *   end_pos  int32 [B]          valid cache length of each row
+ *   topk_idx int32 [B,K]        selected positions (see index semantics)
+ *   wkv_b    bf16 [128*256,512]
+ *   scale    softmax scale applied to the summed latent+rotary score
+ *            (192^-0.5 for the pages' model, times mscale^2 when extended)
+ *   out      bf16 [B,128,128]   per-head output before the output projection
+ *   workspace / workspace_bytes  device scratch, 256-byte aligned, at least
+ *            mla_sparse_decode_workspace_size(B, K, S_max) bytes
+ *   lse_out  optional f32 [B,128]: natural-log sum of exp(scaled score) over
+ *            the selected positions (NULL = not written)
+ *   d_status optional device int: receives MLA_ERR_DEVICE_TIMEOUT if a device
+ *            wait times out (NULL = not written; never cleared by the library)
+ * Returns an mla_status.
+ */
+int mla_sparse_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                      const int32_t* end_pos, const int32_t* topk_idx, const void* wkv_b, float scale, void* out,
+                      int B, int K, int S_max, void* workspace, size_t workspace_bytes, float* lse_out,
+                      int* d_status, cudaStream_t stream);
+
+/*
+ * Step "absorb" alone (model.py 595):
+ *   q_lat[b,h,c] = bf16( sum_d q_nope[b,h,d] * wkv_b[h*256 + d, c] )
+ *   q_nope bf16 [B,128,128], wkv_b bf16 [128*256,512], q_lat bf16 [B,128,512].
+ */
+int mla_absorb_q(const void* q_nope, const void* wkv_b, void* q_lat, int B, cudaStream_t stream);
+
+/*
+ * Steps "scores" .. "mix" for every (row, split) (model.py 596-605), the
+ * key positions of row b being split into `n_split` contiguous ranges of index
+ * slots:
+ *   o_part[b,s,h,:]  f32 [B,n_split,128,512]  softmax-normalised mix of the
+ *                    cached latents over the valid positions of split s
+ *   lse_part[b,s,h]  f32 [B,n_split,128]      log-sum-exp of the split's
+ *                    scaled scores (-inf when the split has no valid index)
+ *   q_lat bf16 [B,128,512] (from mla_absorb_q), the other inputs as above.
+ * n_split must equal mla_num_splits(B, K).
+ */
+int mla_sparse_attend(const void* q_lat, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                      const int32_t* end_pos, const int32_t* topk_idx, float scale, float* o_part,
+                      float* lse_part, int B, int K, int S_max, int n_split, int* d_status, cudaStream_t stream);
+
+/*
+ * Steps "combine" and "value-up" (model.py 605-606):
+ *   O~[b,h,:] = sum_s exp(lse_part[b,s,h] - L) o_part[b,s,h,:],
+ *   L = log sum_s exp(lse_part[b,s,h]),
+ *   out[b,h,e] = bf16( sum_c bf16(O~[b,h,c]) * wkv_b[h*256 + 128 + e, c] ),
+ *   lse_out[b,h] = L (optional).
+ */
+int mla_combine_value_up(const float* o_part, const float* lse_part, const void* wkv_b, void* out,
+                         float* lse_out, int B, int n_split, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_SPARSE_DECODE_H */

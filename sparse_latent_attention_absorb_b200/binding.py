@@ -1,0 +1,186 @@
+"""ctypes binding of ``libmla_sparse_decode.so`` (see include/mla_sparse_decode.h).
+
+Argument marshalling only: these functions check shapes, dtypes and devices of
+torch tensors, pass their device pointers and the current CUDA stream to the
+C ABI, and raise on a non-zero status.  Every step of the decode runs in the
+library's sm_100a kernels; there is no fallback path.  If the library has not
+been built, loading it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .build import LIB_PATH
+
+H, D_NOPE, D_ROPE, D_LAT, D_V = 128, 128, 64, 512, 128
+
+STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_WORKSPACE", 3: "MLA_ERR_CUDA",
+          4: "MLA_ERR_DEVICE_TIMEOUT", 5: "MLA_ERR_BAD_INDEX", 6: "MLA_ERR_UNSUPPORTED"}
+
+# Every symbol the public header declares.
+EXPORTS = ("mla_status_string", "mla_num_splits", "mla_sparse_decode_workspace_size", "mla_sparse_decode",
+           "mla_absorb_q", "mla_sparse_attend", "mla_combine_value_up")
+
+_lib = None
+
+
+class MLAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+def load_library():
+    """Load the CUDA library (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"CUDA library not built: {LIB_PATH} (run sparse_latent_attention_absorb_b200.build)")
+    lib = ctypes.CDLL(LIB_PATH)
+    p, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.mla_status_string.restype = ctypes.c_char_p
+    lib.mla_status_string.argtypes = [i]
+    lib.mla_num_splits.restype = i
+    lib.mla_num_splits.argtypes = [i, i]
+    lib.mla_sparse_decode_workspace_size.restype = sz
+    lib.mla_sparse_decode_workspace_size.argtypes = [i, i, i]
+    lib.mla_sparse_decode.restype = i
+    lib.mla_sparse_decode.argtypes = [p, p, p, p, p, p, p, f, p, i, i, i, p, sz, p, p, p]
+    lib.mla_absorb_q.restype = i
+    lib.mla_absorb_q.argtypes = [p, p, p, i, p]
+    lib.mla_sparse_attend.restype = i
+    lib.mla_sparse_attend.argtypes = [p, p, p, p, p, p, f, p, p, i, i, i, i, p, p]
+    lib.mla_combine_value_up.restype = i
+    lib.mla_combine_value_up.argtypes = [p, p, p, p, p, i, i, p]
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(t: torch.Tensor, name: str, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _raise(rc: int, where: str):
+    if rc != 0:
+        raise MLAError(rc, where)
+
+
+def num_splits(B: int, K: int) -> int:
+    return int(load_library().mla_num_splits(B, K))
+
+
+def workspace_size(B: int, K: int, S_max: int) -> int:
+    return int(load_library().mla_sparse_decode_workspace_size(B, K, S_max))
+
+
+def mla_sparse_decode(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, scale, out=None, workspace=None,
+                      lse_out=None, d_status=None, stream=None):
+    """The whole decode step; returns ``out`` (bf16 [B,128,128])."""
+    lib = load_library()
+    B = q_nope.shape[0]
+    S_max = kv_cache.shape[1]
+    K = topk_idx.shape[1]
+    bf = torch.bfloat16
+    _check(q_nope, "q_nope", bf, (B, H, D_NOPE))
+    _check(q_pe, "q_pe", bf, (B, H, D_ROPE))
+    _check(kv_cache, "kv_cache", bf, (B, S_max, D_LAT))
+    _check(pe_cache, "pe_cache", bf, (B, S_max, D_ROPE))
+    _check(end_pos, "end_pos", torch.int32, (B,))
+    _check(topk_idx, "topk_idx", torch.int32, (B, K))
+    _check(wkv_b, "wkv_b", bf, (H * (D_NOPE + D_V), D_LAT))
+    if out is None:
+        out = torch.empty((B, H, D_V), dtype=bf, device=q_nope.device)
+    _check(out, "out", bf, (B, H, D_V))
+    if lse_out is not None:
+        _check(lse_out, "lse_out", torch.float32, (B, H))
+    if d_status is not None:
+        _check(d_status, "d_status", torch.int32, (1,))
+    need = workspace_size(B, K, S_max)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_nope.device)
+    _check(workspace, "workspace", torch.uint8)
+    rc = lib.mla_sparse_decode(_ptr(q_nope), _ptr(q_pe), _ptr(kv_cache), _ptr(pe_cache), _ptr(end_pos),
+                               _ptr(topk_idx), _ptr(wkv_b), float(scale), _ptr(out), B, K, S_max, _ptr(workspace),
+                               workspace.numel(), _ptr(lse_out), _ptr(d_status), _stream(stream))
+    _raise(rc, "mla_sparse_decode")
+    return out
+
+
+def mla_absorb_q(q_nope, wkv_b, q_lat=None, stream=None):
+    lib = load_library()
+    B = q_nope.shape[0]
+    bf = torch.bfloat16
+    _check(q_nope, "q_nope", bf, (B, H, D_NOPE))
+    _check(wkv_b, "wkv_b", bf, (H * (D_NOPE + D_V), D_LAT))
+    if q_lat is None:
+        q_lat = torch.empty((B, H, D_LAT), dtype=bf, device=q_nope.device)
+    _check(q_lat, "q_lat", bf, (B, H, D_LAT))
+    _raise(lib.mla_absorb_q(_ptr(q_nope), _ptr(wkv_b), _ptr(q_lat), B, _stream(stream)), "mla_absorb_q")
+    return q_lat
+
+
+def mla_sparse_attend(q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, scale, o_part=None, lse_part=None,
+                      d_status=None, stream=None):
+    """Per-split partial outputs; returns (o_part [B,S,128,512] f32, lse_part [B,S,128] f32)."""
+    lib = load_library()
+    B, S_max, K = q_lat.shape[0], kv_cache.shape[1], topk_idx.shape[1]
+    n_split = num_splits(B, K)
+    bf = torch.bfloat16
+    _check(q_lat, "q_lat", bf, (B, H, D_LAT))
+    _check(q_pe, "q_pe", bf, (B, H, D_ROPE))
+    _check(kv_cache, "kv_cache", bf, (B, S_max, D_LAT))
+    _check(pe_cache, "pe_cache", bf, (B, S_max, D_ROPE))
+    _check(end_pos, "end_pos", torch.int32, (B,))
+    _check(topk_idx, "topk_idx", torch.int32, (B, K))
+    dev = q_lat.device
+    if o_part is None:
+        o_part = torch.empty((B, n_split, H, D_LAT), dtype=torch.float32, device=dev)
+    if lse_part is None:
+        lse_part = torch.empty((B, n_split, H), dtype=torch.float32, device=dev)
+    _check(o_part, "o_part", torch.float32, (B, n_split, H, D_LAT))
+    _check(lse_part, "lse_part", torch.float32, (B, n_split, H))
+    rc = lib.mla_sparse_attend(_ptr(q_lat), _ptr(q_pe), _ptr(kv_cache), _ptr(pe_cache), _ptr(end_pos),
+                               _ptr(topk_idx), float(scale), _ptr(o_part), _ptr(lse_part), B, K, S_max, n_split,
+                               _ptr(d_status), _stream(stream))
+    _raise(rc, "mla_sparse_attend")
+    return o_part, lse_part
+
+
+def mla_combine_value_up(o_part, lse_part, wkv_b, out=None, lse_out=None, stream=None):
+    lib = load_library()
+    B, n_split = o_part.shape[0], o_part.shape[1]
+    bf = torch.bfloat16
+    _check(o_part, "o_part", torch.float32, (B, n_split, H, D_LAT))
+    _check(lse_part, "lse_part", torch.float32, (B, n_split, H))
+    _check(wkv_b, "wkv_b", bf, (H * (D_NOPE + D_V), D_LAT))
+    if out is None:
+        out = torch.empty((B, H, D_V), dtype=bf, device=o_part.device)
+    _check(out, "out", bf, (B, H, D_V))
+    if lse_out is not None:
+        _check(lse_out, "lse_out", torch.float32, (B, H))
+    rc = lib.mla_combine_value_up(_ptr(o_part), _ptr(lse_part), _ptr(wkv_b), _ptr(out), _ptr(lse_out), B, n_split,
+                                  _stream(stream))
+    _raise(rc, "mla_combine_value_up")
+    return out

@@ -1,0 +1,299 @@
+// Host side of the sparse MLA decode C ABI (see include/mla_sparse_decode.h):
+// argument validation, key-split planning, TMA tensor-map encoding and the
+// launches of the three sm_100a kernels on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.cuh"
+#include "mla_sparse_decode.h"
+
+namespace {
+
+using namespace mla;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- device info
+
+struct DeviceInfo {
+  int sm_count = 0;
+  bool sm100 = false;
+  bool configured = false;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
+int current_device(DeviceInfo** info) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.configured) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    d.sm100 = (major == 10 && minor == 0);
+    d.sm_count = sms;
+    if (d.sm100) {
+      if (cudaFuncSetAttribute(absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAbsorbSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(sparse_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttendSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(combine_value_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCombineSmemBytes) != cudaSuccess)
+        return MLA_ERR_CUDA;
+    }
+    d.configured = true;
+  }
+  *info = &d;
+  return d.sm100 ? MLA_OK : MLA_ERR_UNSUPPORTED;
+}
+
+// SM count used for split planning; 148 (B200) when no device is visible, so
+// that sizing queries also work on a host without a GPU.
+int planning_sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+    return sms;
+  cudaGetLastError();
+  return 148;
+}
+
+// ---------------------------------------------------------------- tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encoder() {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_encode) return MLA_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return MLA_ERR_CUDA;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return MLA_OK;
+}
+
+// wkv_b as a 2-D bf16 tensor [128*256 rows, 512 columns], boxes of
+// 64 columns x 128 rows, 128-byte swizzle.
+int encode_wkv_b(CUtensorMap* m, const void* wkv_b) {
+  cuuint64_t dims[2] = {(cuuint64_t)kDl, (cuuint64_t)kH * kHeadRows};
+  cuuint64_t strides[1] = {(cuuint64_t)kDl * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(wkv_b), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// q_nope as a 3-D bf16 tensor {d: 128, h: 128, b: B}, boxes of
+// 64 d x 1 head x n_tile rows, 128-byte swizzle (rows past B read as zero).
+int encode_q_nope(CUtensorMap* m, const void* q_nope, int B, int n_tile) {
+  cuuint64_t dims[3] = {(cuuint64_t)kDn, (cuuint64_t)kH, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)kDn * 2, (cuuint64_t)kH * kDn * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)n_tile};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q_nope), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- planning
+
+constexpr int kMaxB = 1 << 20;
+constexpr int kMaxK = 1 << 24;
+
+bool sizes_ok(int B, int K, int S_max) { return B >= 1 && B <= kMaxB && K >= 1 && K <= kMaxK && S_max >= 1; }
+
+// Splits of the K index slots of a row: enough (row, split) pairs to give
+// every 2-SM cluster work, never more splits than 32-slot tiles, each split a
+// whole number of tiles.
+void plan_splits(int B, int K, int sm_count, int* n_split, int* span) {
+  const int clusters = sm_count / 2 > 0 ? sm_count / 2 : 1;
+  const int tiles = ceil_div(K, kNt);
+  int want = clusters / B;
+  if (want < 1) want = 1;
+  if (want > tiles) want = tiles;
+  if (want > kCombineMaxSplits) want = kCombineMaxSplits;
+  const int sp = ceil_div(ceil_div(K, want), kNt) * kNt;
+  *span = sp;
+  *n_split = ceil_div(K, sp);
+}
+
+struct WorkspaceLayout {
+  size_t q_lat = 0, o_part = 0, lse_part = 0, total = 0;
+};
+
+WorkspaceLayout workspace_layout(int B, int n_split) {
+  WorkspaceLayout w;
+  size_t off = 0;
+  w.q_lat = off;
+  off = round_up(off + (size_t)B * kH * kDl * 2, 256);
+  w.o_part = off;
+  off = round_up(off + (size_t)B * n_split * kH * kDl * 4, 256);
+  w.lse_part = off;
+  off = round_up(off + (size_t)B * n_split * kH * 4, 256);
+  w.total = off;
+  return w;
+}
+
+int launch_check() { return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+int launch_absorb(const void* q_nope, const void* wkv_b, void* q_lat, int B, int* d_status, cudaStream_t stream) {
+  const int n_tile = B >= kAbsorbNMax ? kAbsorbNMax : ceil_div(B, 16) * 16;
+  CUtensorMap tm_w, tm_q;
+  int rc;
+  if ((rc = encode_wkv_b(&tm_w, wkv_b)) != MLA_OK) return rc;
+  if ((rc = encode_q_nope(&tm_q, q_nope, B, n_tile)) != MLA_OK) return rc;
+  dim3 grid(kDl / 128, kH, ceil_div(B, kAbsorbNMax));
+  absorb_kernel<<<grid, 128, kAbsorbSmemBytes, stream>>>(tm_w, tm_q, static_cast<__nv_bfloat16*>(q_lat), B, n_tile, d_status);
+  return launch_check();
+}
+
+int launch_attend(const void* q_lat, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                  const int32_t* end_pos, const int32_t* topk_idx, float scale, float* o_part, float* lse_part, int B,
+                  int K, int S_max, int n_split, int span, int* d_status, cudaStream_t stream) {
+  const long long ctas = 2LL * B * n_split;
+  if (ctas > 0x7fffffffLL) return MLA_ERR_INVALID_ARG;
+  sparse_attend_kernel<<<(unsigned)ctas, kAttendThreads, kAttendSmemBytes, stream>>>(
+      static_cast<const __nv_bfloat16*>(q_lat), static_cast<const __nv_bfloat16*>(q_pe),
+      static_cast<const __nv_bfloat16*>(kv_cache), static_cast<const __nv_bfloat16*>(pe_cache), end_pos, topk_idx,
+      scale, o_part, lse_part, K, S_max, n_split, span, d_status);
+  return launch_check();
+}
+
+int launch_combine(const float* o_part, const float* lse_part, const void* wkv_b, void* out, float* lse_out, int B,
+                   int n_split, int* d_status, cudaStream_t stream) {
+  const int n_tile = B >= kCombineNMax ? kCombineNMax : ceil_div(B, 16) * 16;
+  CUtensorMap tm_w;
+  int rc;
+  if ((rc = encode_wkv_b(&tm_w, wkv_b)) != MLA_OK) return rc;
+  dim3 grid(kH, ceil_div(B, kCombineNMax));
+  combine_value_up_kernel<<<grid, kCombineThreads, kCombineSmemBytes, stream>>>(
+      tm_w, o_part, lse_part, static_cast<__nv_bfloat16*>(out), lse_out, B, n_split, n_tile, d_status);
+  return launch_check();
+}
+
+int prepare(DeviceInfo** info) {
+  int rc = current_device(info);
+  if (rc != MLA_OK) return rc;
+  return get_encoder();
+}
+
+}  // namespace
+
+// =============================================================================
+// C ABI
+// =============================================================================
+
+extern "C" const char* mla_status_string(int status) {
+  switch (status) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT";
+    case MLA_ERR_BAD_INDEX: return "MLA_ERR_BAD_INDEX";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    default: return "MLA_ERR_UNKNOWN";
+  }
+}
+
+extern "C" int mla_num_splits(int B, int K) {
+  if (!sizes_ok(B, K, 1)) return 0;
+  int n_split = 0, span = 0;
+  plan_splits(B, K, planning_sm_count(), &n_split, &span);
+  return n_split;
+}
+
+extern "C" size_t mla_sparse_decode_workspace_size(int B, int K, int S_max) {
+  if (!sizes_ok(B, K, S_max)) return 0;
+  int n_split = 0, span = 0;
+  plan_splits(B, K, planning_sm_count(), &n_split, &span);
+  return workspace_layout(B, n_split).total;
+}
+
+extern "C" int mla_absorb_q(const void* q_nope, const void* wkv_b, void* q_lat, int B, cudaStream_t stream) {
+  if (!q_nope || !wkv_b || !q_lat || !aligned16(q_nope) || !aligned16(wkv_b) || !aligned16(q_lat)) return MLA_ERR_INVALID_ARG;
+  if (B < 1 || B > kMaxB) return MLA_ERR_INVALID_ARG;
+  DeviceInfo* info = nullptr;
+  int rc = prepare(&info);
+  if (rc != MLA_OK) return rc;
+  return launch_absorb(q_nope, wkv_b, q_lat, B, nullptr, stream);
+}
+
+extern "C" int mla_sparse_attend(const void* q_lat, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                                 const int32_t* end_pos, const int32_t* topk_idx, float scale, float* o_part,
+                                 float* lse_part, int B, int K, int S_max, int n_split, int* d_status,
+                                 cudaStream_t stream) {
+  const void* ptrs[] = {q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, o_part, lse_part};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  if (!sizes_ok(B, K, S_max) || !std::isfinite(scale)) return MLA_ERR_INVALID_ARG;
+  DeviceInfo* info = nullptr;
+  int rc = prepare(&info);
+  if (rc != MLA_OK) return rc;
+  int want = 0, span = 0;
+  plan_splits(B, K, info->sm_count, &want, &span);
+  if (n_split != want) return MLA_ERR_INVALID_ARG;
+  return launch_attend(q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, scale, o_part, lse_part, B, K, S_max,
+                       n_split, span, d_status, stream);
+}
+
+extern "C" int mla_combine_value_up(const float* o_part, const float* lse_part, const void* wkv_b, void* out,
+                                    float* lse_out, int B, int n_split, cudaStream_t stream) {
+  if (!o_part || !lse_part || !wkv_b || !out) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(o_part) || !aligned16(lse_part) || !aligned16(wkv_b) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
+  if (lse_out && (reinterpret_cast<uintptr_t>(lse_out) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (B < 1 || B > kMaxB || n_split < 1 || n_split > kCombineMaxSplits) return MLA_ERR_INVALID_ARG;
+  DeviceInfo* info = nullptr;
+  int rc = prepare(&info);
+  if (rc != MLA_OK) return rc;
+  return launch_combine(o_part, lse_part, wkv_b, out, lse_out, B, n_split, nullptr, stream);
+}
+
+extern "C" int mla_sparse_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                                 const int32_t* end_pos, const int32_t* topk_idx, const void* wkv_b, float scale,
+                                 void* out, int B, int K, int S_max, void* workspace, size_t workspace_bytes,
+                                 float* lse_out, int* d_status, cudaStream_t stream) {
+  const void* ptrs[] = {q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, out};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  if (lse_out && (reinterpret_cast<uintptr_t>(lse_out) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (!sizes_ok(B, K, S_max) || !std::isfinite(scale)) return MLA_ERR_INVALID_ARG;
+  DeviceInfo* info = nullptr;
+  int rc = prepare(&info);
+  if (rc != MLA_OK) return rc;
+  int n_split = 0, span = 0;
+  plan_splits(B, K, info->sm_count, &n_split, &span);
+  const WorkspaceLayout wl = workspace_layout(B, n_split);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < wl.total)
+    return MLA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* q_lat = ws + wl.q_lat;
+  float* o_part = reinterpret_cast<float*>(ws + wl.o_part);
+  float* lse_part = reinterpret_cast<float*>(ws + wl.lse_part);
+
+  if ((rc = launch_absorb(q_nope, wkv_b, q_lat, B, d_status, stream)) != MLA_OK) return rc;
+  if ((rc = launch_attend(q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, scale, o_part, lse_part, B, K, S_max,
+                          n_split, span, d_status, stream)) != MLA_OK)
+    return rc;
+  return launch_combine(o_part, lse_part, wkv_b, out, lse_out, B, n_split, d_status, stream);
+}

@@ -1,0 +1,115 @@
+"""The C ABI on the host: the library loads and exports every declared symbol,
+status strings, sizing functions and argument validation (which rejects bad
+arguments before touching the GPU).  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_latent_attention_absorb_b200 import binding, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "mla_sparse_decode.h")
+INVALID_ARG, WORKSPACE = 1, 2
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return set(re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", text))
+
+
+def test_header_declarations_match_binding_exports():
+    assert declared_functions() == set(binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_exports_have_c_linkage():
+    out = os.popen(f"nm -D --defined-only {build.LIB_PATH}").read()
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}$", out, flags=re.M), name
+
+
+def test_status_strings(lib):
+    for code, name in binding.STATUS.items():
+        assert lib.mla_status_string(code).decode() == name
+    assert lib.mla_status_string(99).decode() == "MLA_ERR_UNKNOWN"
+
+
+def test_num_splits_properties(lib):
+    assert lib.mla_num_splits(0, 10) == 0 and lib.mla_num_splits(4, 0) == 0
+    for B in (1, 2, 8, 16, 32, 64, 100, 1000):
+        for K in (1, 31, 32, 33, 256, 2048, 8192):
+            n = lib.mla_num_splits(B, K)
+            assert 1 <= n <= max(1, -(-K // 32))
+            assert n <= 128
+            if B >= 74:
+                assert n == 1
+
+
+def test_workspace_size_formula(lib):
+    for B, K in ((1, 256), (8, 2048), (64, 2048), (3, 100)):
+        n = lib.mla_num_splits(B, K)
+        got = lib.mla_sparse_decode_workspace_size(B, K, 4096)
+        need = B * 128 * 512 * 2 + B * n * 128 * 512 * 4 + B * n * 128 * 4
+        assert need <= got <= need + 3 * 256
+    assert lib.mla_sparse_decode_workspace_size(0, 1, 1) == 0
+    assert lib.mla_sparse_decode_workspace_size(1, 1, 0) == 0
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_decode_rejects_bad_arguments_without_a_launch(lib):
+    A = 0x10000  # aligned, never dereferenced: validation fails first
+    good = [_fake(A)] * 7
+
+    def call(ptrs=None, scale=0.07, B=2, K=16, S=32, out=_fake(A), ws=_fake(A), wsb=1 << 30, lse=None, st=None):
+        p = ptrs or good
+        return lib.mla_sparse_decode(*p[:6], p[6], ctypes.c_float(scale), out, B, K, S, ws, wsb, lse, st, None)
+
+    for i in range(7):
+        bad = list(good)
+        bad[i] = None
+        assert call(bad) == INVALID_ARG
+        bad[i] = _fake(A + 8)  # misaligned
+        assert call(bad) == INVALID_ARG
+    assert call(out=None) == INVALID_ARG
+    assert call(B=0) == INVALID_ARG
+    assert call(K=0) == INVALID_ARG
+    assert call(S=0) == INVALID_ARG
+    assert call(scale=float("nan")) == INVALID_ARG
+    assert call(scale=float("inf")) == INVALID_ARG
+    assert call(lse=_fake(A + 2)) == INVALID_ARG
+    assert call(st=_fake(A + 1)) == INVALID_ARG
+
+
+def test_step_entry_points_reject_bad_arguments(lib):
+    A = 0x10000
+    assert lib.mla_absorb_q(None, _fake(A), _fake(A), 4, None) == INVALID_ARG
+    assert lib.mla_absorb_q(_fake(A), _fake(A), _fake(A + 4), 4, None) == INVALID_ARG
+    assert lib.mla_absorb_q(_fake(A), _fake(A), _fake(A), 0, None) == INVALID_ARG
+    args = [_fake(A)] * 6
+    assert lib.mla_sparse_attend(*args, ctypes.c_float(1.0), _fake(A), None, 2, 16, 32, 1, None, None) == INVALID_ARG
+    assert lib.mla_sparse_attend(*args, ctypes.c_float(1.0), _fake(A), _fake(A), 2, 0, 32, 1, None, None) == INVALID_ARG
+    assert lib.mla_combine_value_up(_fake(A), _fake(A), _fake(A), _fake(A), None, 2, 0, None) == INVALID_ARG
+    assert lib.mla_combine_value_up(_fake(A), _fake(A), _fake(A), _fake(A), None, 2, 129, None) == INVALID_ARG
+    assert lib.mla_combine_value_up(_fake(A), None, _fake(A), _fake(A), None, 2, 1, None) == INVALID_ARG
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros((1, 128, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.mla_absorb_q(x, torch.zeros((128 * 256, 512), dtype=torch.bfloat16))

@@ -1,0 +1,253 @@
+"""GPU parity: the sm_100a path through the C ABI against the fp64 oracle on
+the same seeded inputs.
+
+Bounds (the decode step's stated tolerance): bf16 outputs satisfy
+max|out - ref| <= 1e-2 * max|ref| + 1e-3.  Intermediate steps are checked
+against the bound that their own rounding fixes (see each test).  The set of
+positions with non-zero weight is checked bit-exactly by poisoning every
+position that must get zero weight with NaN: the output must not change by a
+single bit.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_latent_attention_absorb_b200 as pkg
+from sparse_latent_attention_absorb_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+DEV = torch.device("cuda:0")
+
+
+def out_bound(ref):
+    return 1e-2 * float(np.max(np.abs(ref))) + 1e-3
+
+
+def to_dev(d):
+    return {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+def gpu_decode(g, lse=True, d_status=None):
+    B = g["q_nope"].shape[0]
+    lse_out = torch.full((B, 128), float("nan"), dtype=torch.float32, device=DEV) if lse else None
+    out = pkg.mla_sparse_decode(g["q_nope"], g["q_pe"], g["kv_cache"], g["pe_cache"], g["end_pos"], g["topk_idx"],
+                                g["wkv_b"], g["scale"], lse_out=lse_out, d_status=d_status)
+    torch.cuda.synchronize()
+    return out, lse_out
+
+
+def run_oracle(d, rows=None, **kw):
+    return oracle.mla_sparse_decode(d["q_nope"], d["q_pe"], d["kv_cache"], d["pe_cache"], d["end_pos"],
+                                    d["topk_idx"], d["wkv_b"], d["scale"], rows=rows, **kw)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from sparse_latent_attention_absorb_b200 import build
+    build.build()
+    pkg.load_library()
+
+
+SMALL = list(wl.SMALL_WORKLOADS) + ["b1_ctx1001_top256"]
+
+
+# ------------------------------------------------------------------ step a1
+
+@pytest.mark.parametrize("B", [1, 5, 16, 64, 130])
+def test_absorb_step_matches_oracle(B):
+    """q_lat = bf16(q_nope . W_UK): fp32 accumulation then one bf16 rounding,
+    so every element is within 2^-8 relative (+ a tiny absolute term for
+    values near zero) of the exact product."""
+    gen = torch.Generator().manual_seed(77 + B)
+    q_nope = torch.randn((B, 128, 128), generator=gen).to(torch.bfloat16)
+    wkv_b = (torch.randn((128 * 256, 512), generator=gen) * 512 ** -0.5).to(torch.bfloat16)
+    q_lat = pkg.mla_absorb_q(q_nope.to(DEV), wkv_b.to(DEV))
+    torch.cuda.synchronize()
+    w_uk = wkv_b.double().view(128, 256, 512)[:, :128, :]
+    ref = torch.einsum("bhd,hdc->bhc", q_nope.double(), w_uk).numpy()
+    got = q_lat.double().cpu().numpy()
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5)
+
+
+# ------------------------------------------------------------------ full path, small cases
+
+@pytest.mark.parametrize("name", SMALL)
+def test_decode_matches_oracle(name):
+    d = wl.generate(name)
+    g = to_dev(d)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out, lse = gpu_decode(g, d_status=status)
+    ref = run_oracle(d)
+    got = out.double().cpu().numpy()
+    assert np.all(np.isfinite(got))
+    err = np.max(np.abs(got - ref.out))
+    assert err <= out_bound(ref.out), (err, out_bound(ref.out))
+    # log-sum-exp: scores carry the bf16 rounding of q_lat (~1e-3 absolute)
+    assert np.max(np.abs(lse.double().cpu().numpy() - ref.lse)) <= 1e-2
+    assert int(status.item()) == 0
+
+
+@pytest.mark.parametrize("name", ["small_b4_ctx600-2k_recent128_top400", "small_b5_ctx40-700_top333"])
+def test_split_outputs_combine_to_oracle_mix(name):
+    """Steps a2-a6: the per-split normalised mixes and log-sum-exps, merged in
+    fp64 on the host, equal the oracle's mixed latent O~ and lse."""
+    d = wl.generate(name)
+    g = to_dev(d)
+    q_lat = pkg.mla_absorb_q(g["q_nope"], g["wkv_b"])
+    o_part, lse_part = pkg.mla_sparse_attend(q_lat, g["q_pe"], g["kv_cache"], g["pe_cache"], g["end_pos"],
+                                             g["topk_idx"], g["scale"])
+    torch.cuda.synchronize()
+    o = o_part.double().cpu().numpy()          # [B, S, H, 512]
+    l = lse_part.double().cpu().numpy()        # [B, S, H]
+    L = np.logaddexp.reduce(l, axis=1)         # [B, H]
+    w = np.exp(l - L[:, None, :])
+    merged = np.einsum("bsh,bshc->bhc", w, o)
+    ref = run_oracle(d, want_o_lat=True)
+    assert np.max(np.abs(L - ref.lse)) <= 1e-2
+    assert np.max(np.abs(merged - ref.o_lat)) <= 1e-2 * np.max(np.abs(ref.o_lat)) + 1e-4
+
+
+def test_combine_step_with_given_partials():
+    """Steps a6-a7 alone on synthetic partials: exact LSE weights, then the
+    W_UV product of the bf16-rounded mix."""
+    gen = torch.Generator().manual_seed(5)
+    B, S = 7, 3  # the combine entry point accepts any split count in [1, 128]
+    o_part = torch.randn((B, S, 128, 512), generator=gen, dtype=torch.float32) * 0.05
+    lse_part = torch.randn((B, S, 128), generator=gen, dtype=torch.float32) * 3
+    lse_part[0, :, 5] = float("-inf")          # a row-head with no valid position
+    wkv_b = (torch.randn((128 * 256, 512), generator=gen) * 512 ** -0.5).to(torch.bfloat16)
+    lse_out = torch.empty((B, 128), dtype=torch.float32, device=DEV)
+    out = pkg.mla_combine_value_up(o_part.to(DEV), lse_part.to(DEV), wkv_b.to(DEV), lse_out=lse_out)
+    torch.cuda.synchronize()
+    l = lse_part.double()
+    L = torch.logsumexp(l, dim=1)
+    wts = torch.exp(l - L[:, None, :]).nan_to_num(0.0)
+    mixed = torch.einsum("bsh,bshc->bhc", wts, o_part.double())
+    w_uv = wkv_b.double().view(128, 256, 512)[:, 128:, :]
+    ref = torch.einsum("bhc,hec->bhe", mixed, w_uv).numpy()
+    got = out.double().cpu().numpy()
+    assert np.max(np.abs(got - ref)) <= out_bound(ref)
+    assert np.all(got[0, 5] == 0.0)
+    lo = lse_out.double().cpu().numpy()
+    assert np.isneginf(lo[0, 5])
+    fin = np.isfinite(L.numpy())
+    assert np.max(np.abs(lo[fin] - L.numpy()[fin])) <= 1e-5 * (1 + np.max(np.abs(L.numpy()[fin])))
+
+
+# ------------------------------------------------------------------ exact zero weights (poison)
+
+@pytest.mark.parametrize("name", ["small_b5_ctx40-700_top333", "small_b2_ctx9000_runs6x37"])
+def test_unselected_positions_get_exactly_zero_weight(name):
+    d = wl.generate(name)
+    g = to_dev(d)
+    clean, clean_lse = gpu_decode(g)
+    # NaN into every cache row that is not selected (including rows >= end_pos)
+    B, S_max = d["kv_cache"].shape[:2]
+    keep = torch.zeros((B, S_max), dtype=torch.bool)
+    for b in range(B):
+        ep = int(d["end_pos"][b])
+        idx = d["topk_idx"][b]
+        idx = idx[(idx >= 0) & (idx < ep)].long()
+        keep[b, idx] = True
+    kv = d["kv_cache"].clone()
+    pe = d["pe_cache"].clone()
+    kv[~keep] = float("nan")
+    pe[~keep] = float("nan")
+    g2 = dict(g, kv_cache=kv.to(DEV), pe_cache=pe.to(DEV))
+    poisoned, poisoned_lse = gpu_decode(g2)
+    assert torch.equal(clean.view(torch.int16), poisoned.view(torch.int16))
+    assert torch.equal(clean_lse, poisoned_lse)
+    assert torch.isfinite(clean.float()).all()
+
+
+def test_index_order_and_padding_placement_do_not_matter():
+    d = wl.generate("small_b4_ctx600-2k_recent128_top400")
+    g = to_dev(d)
+    base, _ = gpu_decode(g)
+    gen = torch.Generator().manual_seed(3)
+    idx = d["topk_idx"].clone()
+    for b in range(idx.shape[0]):
+        idx[b] = idx[b, torch.randperm(idx.shape[1], generator=gen)]
+    shuffled, _ = gpu_decode(dict(g, topk_idx=idx.to(DEV)))
+    ref = run_oracle(d)
+    assert np.max(np.abs(shuffled.double().cpu().numpy() - ref.out)) <= out_bound(ref.out)
+    assert np.max(np.abs(shuffled.double().cpu().numpy() - base.double().cpu().numpy())) <= out_bound(ref.out)
+
+
+def test_rows_without_valid_index_and_out_of_range_entries():
+    d = wl.generate("small_b5_ctx40-700_top333")
+    idx = d["topk_idx"].clone()
+    idx[1] = -1                                       # nothing selected
+    idx[2, :5] = torch.tensor([-7, 10 ** 6, int(d["end_pos"][2]), 704, -1], dtype=torch.int32)
+    d2 = dict(d, topk_idx=idx)
+    out, lse = gpu_decode(to_dev(d2))
+    ref = run_oracle(d2)
+    got = out.double().cpu().numpy()
+    assert np.all(got[1] == 0.0)
+    assert np.all(np.isneginf(lse.cpu().numpy()[1]))
+    assert np.max(np.abs(got - ref.out)) <= out_bound(ref.out)
+
+
+def test_single_selected_position_closed_form():
+    """|T_b| = 1: out[b,h] = W_UV[h] . kv[b,t] whatever the query (up to bf16
+    rounding of the mixed latent, which here is the cached row itself)."""
+    d = wl.generate("small_b2_ctx300_top100")
+    idx = torch.full_like(d["topk_idx"], -1)
+    idx[0, 37] = 123
+    idx[1, 0] = 0
+    d2 = dict(d, topk_idx=idx)
+    out, _ = gpu_decode(to_dev(d2))
+    w_uv = d["wkv_b"].double().view(128, 256, 512)[:, 128:, :]
+    for b, t in ((0, 123), (1, 0)):
+        ref = torch.einsum("hec,c->he", w_uv, d["kv_cache"][b, t].double()).numpy()
+        got = out[b].double().cpu().numpy()
+        assert np.max(np.abs(got - ref)) <= out_bound(ref)
+
+
+def test_repeated_calls_are_deterministic():
+    d = wl.generate("small_b3_ctx1001_top256")
+    g = to_dev(d)
+    a, la = gpu_decode(g)
+    b, lb = gpu_decode(g)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16)) and torch.equal(la, lb)
+
+
+def test_workspace_too_small_is_rejected():
+    d = wl.generate("small_b2_ctx300_top100")
+    g = to_dev(d)
+    B, K, S = d["q_nope"].shape[0], d["topk_idx"].shape[1], d["kv_cache"].shape[1]
+    ws = torch.empty(pkg.workspace_size(B, K, S) - 256, dtype=torch.uint8, device=DEV)
+    with pytest.raises(pkg.MLAError) as e:
+        pkg.mla_sparse_decode(g["q_nope"], g["q_pe"], g["kv_cache"], g["pe_cache"], g["end_pos"], g["topk_idx"],
+                              g["wkv_b"], g["scale"], workspace=ws)
+    assert e.value.code == 2
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled rows
+
+FULL = ["b8_ctx4096_top2048", "b32_ctx2k-8k_recent512_top2048", "b64_ctx1k-32k_top2048",
+        "b16_ctx131072_runs32x64", "b16_ctx8192_dense"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workloads_sampled_rows(name):
+    """The benchmark's launch configuration at the full sizes; the oracle
+    recomputes a sample of batch rows (all 128 heads each)."""
+    d = wl.generate(name)
+    g = to_dev(d)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out, lse = gpu_decode(g, d_status=status)
+    B = d["q_nope"].shape[0]
+    rows = sorted({0, B - 1, B // 2, (7 * B) // 11})
+    ref = run_oracle(d, rows=rows)
+    got = out.double().cpu().numpy()[rows]
+    assert np.all(np.isfinite(out.float().cpu().numpy()))
+    assert np.max(np.abs(got - ref.out)) <= out_bound(ref.out)
+    assert np.max(np.abs(lse.double().cpu().numpy()[rows] - ref.lse)) <= 1e-2
+    assert int(status.item()) == 0
+    del g
+    torch.cuda.empty_cache()
