@@ -133,55 +133,86 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 // sparse_attend_kernel
 //
 // One 2-CTA cluster per (batch row b, key split s).  CTA rank r owns latent
-// columns [256r, 256r+256) and rotary columns [32r, 32r+32):
-//   * it gathers, for every selected position t of the split, kv[b,t,its 256]
-//     and pe[b,t,its 32] into shared memory (cp.async, 128B-swizzled rows);
+// columns [256r, 256r+256) and rotary columns [32r, 32r+32) of the score:
+//   * its half of the absorbed query is an MMA operand: q_lat[b, :, its 256]
+//     in TMEM (bf16 pairs), q_pe[b, :, its 32] in shared memory;
+//   * for every selected position t of the split, four gather warps copy
+//     kv[b,t,its 256] (128B-swizzled rows) and pe[b,t,its 32] (64B-swizzled
+//     rows) into a ring of 64-position tiles (cp.async, 16 bytes per lane);
+//     padding positions are zero-filled without a read;
 //   * QK: S_r[h,t] = q_lat[h, its 256] . kv[t, its 256] + q_pe[h, its 32] .
-//     pe[t, its 32]  -- a split-K half of the 576-wide score, M = 128 heads;
-//   * the two halves are exchanged through distributed shared memory, so both
-//     CTAs hold the full score S = S_0 + S_1 (bitwise identical in both);
-//   * online softmax with a lazily updated running maximum (O is rescaled
-//     only when the maximum grows by more than 2^8); P (bf16) goes to TMEM;
+//     pe[t, its 32]  -- a split-K half of the 576-wide score, M = 128 heads,
+//     N = 64 positions, into a TMEM score buffer;
+//   * four exchange warps swap the halves through distributed shared memory
+//     (st.async with transaction counts on the receiver's mbarrier) and write
+//     the full score S = S_0 + S_1 back into the buffer (bitwise identical in
+//     both CTAs: fp32 addition commutes), one tile ahead of the softmax;
+//   * eight softmax warps: online softmax with a lazily updated running
+//     maximum (O is rescaled only when the maximum grows by more than 2^8);
+//     P (bf16) is written into the same TMEM buffer over the scores;
 //   * PV: O_r[h, its 256] += P[h,t] . kv[t, its 256]  (A = P from TMEM,
-//     B = the same gathered rows read M/N-major).
+//     B = the same gathered rows read M/N-major).  tcgen05.mma operations of
+//     one CTA execute in issue order, so QK(j+2) issued after PV(j) may
+//     overwrite the buffer that holds P(j).
 // The split's normalised O and its log-sum-exp go to o_part / lse_part.
 //
-// Warp roles (288 threads): warps 0-3 softmax (thread i <-> TMEM lane i =
-// head i), warp 4 TMEM allocation + MMA issue, warps 5-8 gather.
+// Warp roles (544 threads): warps 0-7 softmax (warps w and w+4 share TMEM
+// lanes 32(w%4).. and take positions 0-31 / 32-63 of every tile); warps 8-11
+// score exchange (lanes 32(w%4).., all 64 positions); warp 12 TMEM
+// allocation + MMA issue; warps 13-16 gather (one stage each).
 // =============================================================================
-constexpr int kNt = 32;                            // positions per tile
-constexpr int kStages = 5;                         // gathered tile ring
-constexpr int kLag = kStages - 2;                  // cp.async groups in flight before a tile is published
-constexpr int kKB = 5;                             // 128-byte K blocks per row: 4 latent + 1 rotary (half used)
-constexpr int kQBytes = kKB * kH * 128;            // 80 KB
-constexpr int kStageBytes = kKB * kNt * 128;       // 20 KB
-constexpr int kXBytes = (kNt / 4) * kH * 16;       // 16 KB: one exchanged score tile (f32)
-constexpr int kOffQ = 0;
-constexpr int kOffStage = kOffQ + kQBytes;
+constexpr int kNt = 64;                            // positions per tile
+constexpr int kStages = 4;                         // gathered tile ring
+constexpr int kXBufs = 2;                          // score-exchange buffers
+constexpr int kLatBlock = kNt * 128;               // one 64-column latent block of a tile (8 KB)
+constexpr int kStageBytes = 4 * kLatBlock + kNt * 64;  // 4 latent blocks + the rotary block: 36 KB
+constexpr int kQpeBytes = kH * 64;                 // 8 KB
+constexpr int kXBytes = (kNt / 4) * kH * 16;       // 32 KB: one exchanged score tile (f32)
+constexpr int kRedBytes = 2 * 2 * kH * 4;          // row maxima / sums shared by warp pairs
+constexpr int kOffStage = 0;
 constexpr int kOffX = kOffStage + kStages * kStageBytes;
-constexpr int kOffBar = kOffX + 2 * kXBytes;
+constexpr int kOffQpe = kOffX + kXBufs * kXBytes;
+constexpr int kOffRed = kOffQpe + kQpeBytes;
+constexpr int kOffBar = kOffRed + kRedBytes;
 constexpr int kAttendSmemBytes = kOffBar + 256 + kSmemAlignPad;
-constexpr int kAttendThreads = 288;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kXchgWarp0 = 8;
+constexpr int kXchgWarps = 4;
+constexpr int kMmaWarp = 12;
+constexpr int kGatherWarp0 = 13;
+constexpr int kGatherWarps = kStages;  // gather warp g always fills stage g
+constexpr int kAttendThreads = 32 * (kGatherWarp0 + kGatherWarps);  // 544
 // TMEM columns
-constexpr uint32_t kColS = 0;     // two score buffers of kNt columns
-constexpr uint32_t kColP = 64;    // two P buffers of kNt/2 columns (bf16 pairs)
-constexpr uint32_t kColO = 256;   // 256 columns of O
+constexpr uint32_t kColS = 0;     // two score buffers of kNt f32 columns; P (bf16 pairs) over the first kNt/2
+constexpr uint32_t kColQ = 128;   // 128 columns: 256 bf16 of the latent query half
+constexpr uint32_t kColO = 256;   // 256 f32 columns of O
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-static_assert(kOffStage % 1024 == 0 && kStageBytes % 1024 == 0 && kOffX % 1024 == 0, "swizzle atoms");
+static_assert(kStageBytes % 1024 == 0 && kOffX % 1024 == 0 && kOffQpe % 1024 == 0, "swizzle atoms");
 static_assert(kAttendSmemBytes <= 232448, "shared memory");
-static_assert(kLag >= 1, "pipeline");
+static_assert(kColS + 2 * kNt <= kColQ && kColQ + 128 <= kColO, "TMEM map");
+// Exchange buffers: the exchange warps of a CTA push tile t into the peer's
+// buffer t mod 2 after they have received the peer's push of tile t-1, which
+// every peer exchange warp issued after it had read tile t-2 from that same
+// buffer.
+static_assert(kXBufs >= 2, "score exchange reuse distance");
+// Each gather warp owns one stage (tiles g, g+kStages, ...), so every wait on
+// a stage's kv_empty barrier is exactly one phase after the warp's previous
+// wait on it; with fewer stages than warps a waiter could run two phases
+// ahead of the barrier, where a parity test cannot tell the phases apart.
+static_assert(kGatherWarps == kStages, "one stage per gather warp");
+static_assert(kXchgWarp0 % 4 == 0 && kXchgWarps == 4, "exchange warps cover the four TMEM lane quarters");
 
 struct AttendBars {
-  uint64_t q_full;
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
-  uint64_t s_full[2];
-  uint64_t s_empty[2];
-  uint64_t p_full[2];
-  uint64_t o_done;
-  uint64_t x_full[2];
-  uint64_t x_free[2];
+  uint64_t q_full;              // softmax warps (8 arrivals) after storing Q
+  uint64_t kv_full[kStages];    // the tile's gather warp (1 arrival) once its copies landed
+  uint64_t kv_empty[kStages];   // MMA commit after PV of the tile
+  uint64_t s_full[2];           // MMA commit after QK: partial scores in the buffer
+  uint64_t s_sum[2];            // exchange warps (4) after writing the full scores back
+  uint64_t p_full[2];           // softmax warps (8) after writing P over the scores
+  uint64_t p_free[2];           // MMA commit after PV of the tile: O stable
+  uint64_t x_full[kXBufs];      // 1 local arrival + kXBytes from the peer's st.async
+  uint32_t vmask[kStages][2];   // valid positions of the tile in each stage (bit n of word n/32)
   uint32_t tmem_addr;
   int abort_flag;
 };
@@ -192,6 +223,39 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// Optional pipeline trace (compile with -DMLA_TRACE): per-tile clock64()
+// stamps of each pipeline event for the first cluster of a launch, read back
+// with mla_trace_fetch().  Compiled out by default.
+enum TraceEvent {
+  kTrGatherIssue = 0,  // gather warp: copies of the tile issued
+  kTrGatherLanded,     // gather warp: copies landed, tile published
+  kTrQkStart,          // MMA thread: QK of the tile starts issuing
+  kTrQkIssued,         // MMA thread: QK of the tile issued and committed
+  kTrPvStart,          // MMA thread: PV of the tile starts issuing
+  kTrPvIssued,         // MMA thread: PV of the tile issued and committed
+  kTrXStart,           // exchange warp 8: partial scores of the tile available
+  kTrXPushed,          // exchange warp 8: partial scores pushed to the peer
+  kTrXArrived,         // exchange warp 8: peer's partial scores observed
+  kTrXSummed,          // exchange warp 8: full scores written back
+  kTrSmStart,          // softmax warp 0: full scores of the tile available
+  kTrMaxShared,        // softmax warp 0: tile maximum shared with its partner warp
+  kTrPWritten,         // softmax warp 0: P of the tile written, p_full arrived
+  kTrEvents
+};
+constexpr int kTraceTiles = 512;
+#ifdef MLA_TRACE
+__device__ long long g_mla_trace[2 * kTrEvents * kTraceTiles];
+#define MLA_TRACE_STAMP(ev, tile)                                                               \
+  do {                                                                                           \
+    if ((blockIdx.x >> 1) == 0 && (tile) < kTraceTiles)                                          \
+      g_mla_trace[(rank * kTrEvents + (ev)) * kTraceTiles + (tile)] = clock64();                 \
+  } while (0)
+#else
+#define MLA_TRACE_STAMP(ev, tile) \
+  do {                            \
+  } while (0)
+#endif
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttendThreads, 1)
 sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat16* __restrict__ q_pe,
@@ -212,251 +276,358 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
   const int n_tiles = k_end > k_begin ? (k_end - k_begin + kNt - 1) / kNt : 0;
   int ep = end_pos[b];
   ep = ep < 0 ? 0 : (ep > S_max ? S_max : ep);
+  const int32_t* idx_row = topk_idx + (size_t)b * K;
 
-  const uint32_t sQ = smem_u32(smem + kOffQ);
   const uint32_t sStage = smem_u32(smem + kOffStage);
   const uint32_t sX = smem_u32(smem + kOffX);
+  const uint32_t sQpe = smem_u32(smem + kOffQpe);
+  float* red = reinterpret_cast<float*>(smem + kOffRed);  // [tile parity][half][head]
   AttendBars* bars = reinterpret_cast<AttendBars*>(smem + kOffBar);
   const AbortState ab{&bars->abort_flag, d_status};
 
   if (tid == 0) {
     bars->abort_flag = 0;
-    mbar_init(smem_u32(&bars->q_full), 128);
+    mbar_init(smem_u32(&bars->q_full), kSoftmaxWarps);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(smem_u32(&bars->kv_full[i]), 128);
+      mbar_init(smem_u32(&bars->kv_full[i]), 1);
       mbar_init(smem_u32(&bars->kv_empty[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars->s_full[i]), 1);
-      mbar_init(smem_u32(&bars->s_empty[i]), 128);
-      mbar_init(smem_u32(&bars->p_full[i]), 128);
-      mbar_init(smem_u32(&bars->x_full[i]), 128);
-      mbar_init(smem_u32(&bars->x_free[i]), 128);
+      mbar_init(smem_u32(&bars->s_sum[i]), kXchgWarps);
+      mbar_init(smem_u32(&bars->p_full[i]), kSoftmaxWarps);
+      mbar_init(smem_u32(&bars->p_free[i]), 1);
     }
-    mbar_init(smem_u32(&bars->o_done), 1);
+    for (int i = 0; i < kXBufs; ++i) {
+      mbar_init(smem_u32(&bars->x_full[i]), 1);
+      mbar_arrive_expect_tx(smem_u32(&bars->x_full[i]), kXBytes);  // armed for tiles 0..kXBufs-1
+    }
     fence_mbarrier_init_cluster();
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(&bars->tmem_addr), 512);
     tmem_relinquish();
   }
   tc_fence_before();
-  cluster_sync();  // barriers of both CTAs initialised before any remote arrive
+  cluster_sync();  // barriers of both CTAs initialised before any remote access
   tc_fence_after();
   const uint32_t tmem = bars->tmem_addr;
 
-  if (warp >= 5) {
+  if (warp >= kGatherWarp0) {
     // ------------------------------------------------------------ gather
-    const int ptid = tid - 160;  // 0..127
-    const int pw = warp - 5;     // 0..3, 8 positions of each tile
-    // Q half: q_lat[b, h, 256r + 8q .. +8] and q_pe[b, h, 32r + 8q .. +8]
-    for (int i = ptid; i < kH * 32; i += 128) {
-      const int hh = i >> 5, q = i & 31;
-      const uint32_t dst = sQ + (q >> 3) * (kH * 128) + sw128_offset(hh, q & 7);
-      cp_async_16(dst, q_lat + ((size_t)b * kH + hh) * kDl + rank * 256 + q * 8, 16);
-    }
-    for (int i = ptid; i < kH * 4; i += 128) {
-      const int hh = i >> 2, q = i & 3;
-      const uint32_t dst = sQ + 4 * (kH * 128) + sw128_offset(hh, q);
-      cp_async_16(dst, q_pe + ((size_t)b * kH + hh) * kDr + rank * 32 + q * 8, 16);
-    }
-    cp_async_commit();
-
+    // Gather warp g owns stage g and tiles g, g+4, g+8, ...; lane l handles
+    // positions l and l+32 of a tile.  Latent: one position per instruction
+    // (32 lanes x 16 bytes = this CTA's 256 columns); rotary: eight positions
+    // per instruction (this CTA's 32 columns).  A tile is published
+    // (kv_full) as soon as its own copies have landed.
+    const int g = warp - kGatherWarp0;
     const __nv_bfloat16* kv_row0 = kv_cache + (size_t)b * S_max * kDl + rank * 256;
     const __nv_bfloat16* pe_row0 = pe_cache + (size_t)b * S_max * kDr + rank * 32;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int st = j % kStages;
+    auto load_idx = [&](int t, int half) -> int {
+      int v = -1;
+      if (t < n_tiles) {
+        const int k = k_begin + t * kNt + half * 32 + lane;
+        if (k < k_end) v = __ldg(idx_row + k);
+      }
+      return (v >= 0 && v < ep) ? v : -1;
+    };
+    auto gather_tile = [&](int j, int idx0, int idx1) {
+      const int st = g;
       if (j >= kStages) wait(smem_u32(&bars->kv_empty[st]), ((j / kStages) - 1) & 1, ab);
       const uint32_t stage = sStage + st * kStageBytes;
-      // lanes 0..7 fetch the indices of this warp's 8 positions
-      int idx = -1;
-      if (lane < 8) {
-        const int k = k_begin + j * kNt + pw * 8 + lane;
-        if (k < k_end) idx = topk_idx[(size_t)b * K + k];
+#pragma unroll 8
+      for (int n = 0; n < kNt; ++n) {
+        const int pos = __shfl_sync(0xffffffffu, n < 32 ? idx0 : idx1, n & 31);
+        const size_t p = pos >= 0 ? (size_t)pos : 0;
+        const uint32_t dst = stage + (lane >> 3) * kLatBlock + sw128_offset(n, lane & 7);
+        cp_async_16(dst, kv_row0 + p * kDl + lane * 8, pos >= 0 ? 16u : 0u);
       }
 #pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const int n = pw * 8 + t;  // row of the tile
-        const int pos = __shfl_sync(0xffffffffu, idx, t);
-        const bool valid = pos >= 0 && pos < ep;
-        const size_t p = valid ? (size_t)pos : 0;
-        // latent: lane l copies 16 bytes = 8 columns [8l, 8l+8) of the half
-        {
-          const uint32_t dst = stage + (lane >> 3) * (kNt * 128) + sw128_offset(n, lane & 7);
-          cp_async_16(dst, kv_row0 + p * kDl + lane * 8, valid ? 16u : 0u);
-        }
-        if (lane < 4) {
-          const uint32_t dst = stage + 4 * (kNt * 128) + sw128_offset(n, lane);
-          cp_async_16(dst, pe_row0 + p * kDr + lane * 8, valid ? 16u : 0u);
-        }
+      for (int q = 0; q < kNt / 8; ++q) {
+        const int n = q * 8 + (lane >> 2), c = lane & 3;
+        const int pos = __shfl_sync(0xffffffffu, q < 4 ? idx0 : idx1, n & 31);
+        const size_t p = pos >= 0 ? (size_t)pos : 0;
+        const uint32_t dst = stage + 4 * kLatBlock + sw64_offset(n, c);
+        cp_async_16(dst, pe_row0 + p * kDr + c * 8, pos >= 0 ? 16u : 0u);
       }
       cp_async_commit();
-      if (j >= kLag) {
-        cp_async_wait_group<kLag>();
-        fence_proxy_async_smem();
-        const int jt = j - kLag;
-        if (jt == 0) mbar_arrive(smem_u32(&bars->q_full));
-        mbar_arrive(smem_u32(&bars->kv_full[jt % kStages]));
+      if (lane == 0) MLA_TRACE_STAMP(kTrGatherIssue, j);
+      const uint32_t valid0 = __ballot_sync(0xffffffffu, idx0 >= 0);
+      const uint32_t valid1 = __ballot_sync(0xffffffffu, idx1 >= 0);
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        bars->vmask[st][0] = valid0;  // published by the arrival below
+        bars->vmask[st][1] = valid1;
+        mbar_arrive(smem_u32(&bars->kv_full[st]));
+        MLA_TRACE_STAMP(kTrGatherLanded, j);
+      }
+    };
+    // this warp's next two tiles, statically indexed (a register copy of a
+    // pending load would wait for the load)
+    int a0 = load_idx(g, 0), a1 = load_idx(g, 1);
+    int b0 = load_idx(g + kStages, 0), b1 = load_idx(g + kStages, 1);
+    for (int j = g; j < n_tiles; j += 2 * kStages) {
+      gather_tile(j, a0, a1);
+      a0 = load_idx(j + 2 * kStages, 0);
+      a1 = load_idx(j + 2 * kStages, 1);
+      if (j + kStages < n_tiles) {
+        gather_tile(j + kStages, b0, b1);
+        b0 = load_idx(j + 3 * kStages, 0);
+        b1 = load_idx(j + 3 * kStages, 1);
       }
     }
-    cp_async_wait_all();
-    fence_proxy_async_smem();
-    for (int jt = n_tiles - kLag < 0 ? 0 : n_tiles - kLag; jt < n_tiles; ++jt) {
-      if (jt == 0) mbar_arrive(smem_u32(&bars->q_full));
-      mbar_arrive(smem_u32(&bars->kv_full[jt % kStages]));
-    }
-    if (n_tiles == 0) mbar_arrive(smem_u32(&bars->q_full));
-  } else if (warp == 4) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
+    // In order: QK(0), QK(1), then for every tile j: PV(j) once P(j) is
+    // written, then QK(j+2) into the buffer P(j) occupied once its rows have
+    // landed.
     if (lane == 0 && n_tiles > 0) {
-      const uint32_t idesc_qk = idesc_bf16_f32(128, kNt, false, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kNt, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+      // Descriptors are built once; an operand at byte offset x from a base
+      // is the base descriptor plus x/16 (start-address field).
+      const uint64_t d_lat = smem_desc_sw128(sStage, 16, 1024);            // QK B, latent, K-major
+      const uint64_t d_pe = smem_desc_sw64(sStage + 4 * kLatBlock, 512);    // QK B, rotary, K-major
+      const uint64_t d_qpe = smem_desc_sw64(sQpe, 512);                     // QK A, rotary, K-major
+      const uint64_t d_v = smem_desc_sw128(sStage, kLatBlock, 1024);        // PV B, latent, N-major
       wait(smem_u32(&bars->q_full), 0, ab);
-      auto issue_pv = [&](int t) {
-        wait(smem_u32(&bars->p_full[t & 1]), (t >> 1) & 1, ab);
+      tc_fence_after();
+      auto issue_qk = [&](int t) {
+        const int st = t % kStages;
+        wait(smem_u32(&bars->kv_full[st]), (t / kStages) & 1, ab);
         tc_fence_after();
-        const uint32_t stage = sStage + (t % kStages) * kStageBytes;
+        MLA_TRACE_STAMP(kTrQkStart, t);
+        const uint64_t dl = d_lat + (uint64_t)((st * kStageBytes) >> 4);
+        const uint64_t dr = d_pe + (uint64_t)((st * kStageBytes) >> 4);
+        const uint32_t dst = tmem + kColS + (t & 1) * kNt;
 #pragma unroll
-        for (int k = 0; k < kNt / 16; ++k) {
-          // B = gathered latent rows read N-major: 16 positions per step,
-          // the four 64-column blocks kNt*128 bytes apart.
-          const uint64_t bdesc = smem_desc_sw128(stage + k * 16 * 128, kNt * 128, 1024);
-          mma_ts(tmem + kColO, tmem + kColP + (t & 1) * (kNt / 2) + k * 8, bdesc, idesc_pv,
-                 (t > 0 || k > 0) ? 1u : 0u);
-        }
-        mma_commit(smem_u32(&bars->kv_empty[t % kStages]));
-        mma_commit(smem_u32(&bars->o_done));
+        for (int k = 0; k < 16; ++k)  // latent: K block k/4, 32 bytes per step
+          mma_ts(dst, tmem + kColQ + k * 8, dl + (uint64_t)(((k >> 2) * kLatBlock + (k & 3) * 32) >> 4), idesc_qk,
+                 k > 0 ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < 2; ++k)  // rotary: 32 bytes per step inside the 64-byte rows
+          mma_ss(dst, d_qpe + (uint64_t)((k * 32) >> 4), dr + (uint64_t)((k * 32) >> 4), idesc_qk, 1u);
+        mma_commit(smem_u32(&bars->s_full[t & 1]));
+        MLA_TRACE_STAMP(kTrQkIssued, t);
       };
+      issue_qk(0);
+      if (n_tiles > 1) issue_qk(1);
       for (int j = 0; j < n_tiles; ++j) {
         const int st = j % kStages;
-        wait(smem_u32(&bars->kv_full[st]), (j / kStages) & 1, ab);
-        if (j >= 2) wait(smem_u32(&bars->s_empty[j & 1]), ((j >> 1) - 1) & 1, ab);
+        wait(smem_u32(&bars->p_full[j & 1]), (j >> 1) & 1, ab);
         tc_fence_after();
-        const uint32_t stage = sStage + st * kStageBytes;
+        MLA_TRACE_STAMP(kTrPvStart, j);
+        const uint64_t dv = d_v + (uint64_t)((st * kStageBytes) >> 4);
+        const uint32_t pa = tmem + kColS + (j & 1) * kNt;  // P(j): kNt/2 columns of bf16 pairs
 #pragma unroll
-        for (int k = 0; k < 18; ++k) {
-          const int kb = k < 16 ? (k >> 2) : 4;
-          const int within = (k < 16 ? (k & 3) : (k - 16)) * 32;
-          const uint64_t adesc = smem_desc_sw128(sQ + kb * (kH * 128) + within, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(stage + kb * (kNt * 128) + within, 16, 1024);
-          mma_ss(tmem + kColS + (j & 1) * kNt, adesc, bdesc, idesc_qk, k > 0 ? 1u : 0u);
-        }
-        mma_commit(smem_u32(&bars->s_full[j & 1]));
-        if (j >= 1) issue_pv(j - 1);
+        for (int k = 0; k < kNt / 16; ++k)  // 16 positions per step
+          mma_ts(tmem + kColO, pa + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+        mma_commit(smem_u32(&bars->kv_empty[st]));
+        mma_commit(smem_u32(&bars->p_free[j & 1]));
+        MLA_TRACE_STAMP(kTrPvIssued, j);
+        if (j + 2 < n_tiles) issue_qk(j + 2);
       }
-      issue_pv(n_tiles - 1);
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------ softmax
-    const int i = tid;  // head
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const float c2 = scale * 1.4426950408889634f;  // scores to log2 units
-    float m_used = -INFINITY, l_sum = 0.f;
-    uint32_t x_peer[2], xfull_peer[2], xfree_peer[2];
-    for (int u = 0; u < 2; ++u) {
+  } else if (warp >= kXchgWarp0) {
+    // ------------------------------------------------------------ exchange
+    const int qd = warp & 3;
+    const int i = qd * 32 + lane;  // head
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    const bool leader = (warp == kXchgWarp0 && lane == 0);
+    uint32_t x_peer[kXBufs], xfull_peer[kXBufs];
+#pragma unroll
+    for (int u = 0; u < kXBufs; ++u) {
       x_peer[u] = cluster_map(sX + u * kXBytes, peer);
       xfull_peer[u] = cluster_map(smem_u32(&bars->x_full[u]), peer);
-      xfree_peer[u] = cluster_map(smem_u32(&bars->x_free[u]), peer);
     }
     for (int j = 0; j < n_tiles; ++j) {
-      const int u = j & 1;
-      // validity of the tile's positions (same in every softmax warp)
-      int pos = -1;
-      {
-        const int k = k_begin + j * kNt + lane;
-        if (k < k_end) pos = topk_idx[(size_t)b * K + k];
-      }
-      const uint32_t vmask = __ballot_sync(0xffffffffu, pos >= 0 && pos < ep);
-
-      wait(smem_u32(&bars->s_full[u]), (j >> 1) & 1, ab);
+      const int u = j % kXBufs;
+      const uint32_t sbuf = tmem + lane_base + kColS + (j & 1) * kNt;
+      wait(smem_u32(&bars->s_full[j & 1]), (j >> 1) & 1, ab);
       tc_fence_after();
-      uint32_t sv[32];
-      tmem_ld32(tmem + lane_base + kColS + u * kNt, sv);
-      tmem_wait_ld();
+      if (leader) MLA_TRACE_STAMP(kTrXStart, j);
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {  // positions [32 h2, 32 h2 + 32)
+        uint32_t sv[32];
+        tmem_ld32(sbuf + 32 * h2, sv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          st_async_v4(x_peer[u] + (uint32_t)(((8 * h2 + q) * kH + i) * 16), sv[4 * q], sv[4 * q + 1],
+                      sv[4 * q + 2], sv[4 * q + 3], xfull_peer[u]);
+      }
+      if (leader) MLA_TRACE_STAMP(kTrXPushed, j);
+      wait(smem_u32(&bars->x_full[u]), (j / kXBufs) & 1, ab);
+      if (leader) {
+        MLA_TRACE_STAMP(kTrXArrived, j);
+        mbar_arrive_expect_tx(smem_u32(&bars->x_full[u]), kXBytes);  // re-arm for tile j + kXBufs
+      }
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t sv[32];
+        tmem_ld32(sbuf + 32 * h2, sv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 o = *reinterpret_cast<const float4*>(smem + kOffX + u * kXBytes + ((8 * h2 + q) * kH + i) * 16);
+          sv[4 * q + 0] = __float_as_uint(__uint_as_float(sv[4 * q + 0]) + o.x);
+          sv[4 * q + 1] = __float_as_uint(__uint_as_float(sv[4 * q + 1]) + o.y);
+          sv[4 * q + 2] = __float_as_uint(__uint_as_float(sv[4 * q + 2]) + o.z);
+          sv[4 * q + 3] = __float_as_uint(__uint_as_float(sv[4 * q + 3]) + o.w);
+        }
+        tmem_st32(sbuf + 32 * h2, sv);
+      }
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&bars->s_empty[u]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->s_sum[j & 1]));
+      if (leader) MLA_TRACE_STAMP(kTrXSummed, j);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int qd = warp & 3;        // TMEM lane quarter
+    const int hf = warp >> 2;       // positions [32hf, 32hf+32) of every tile
+    const int i = qd * 32 + lane;   // head
+    const bool leader = (warp == 0 && lane == 0);
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    const float c2 = scale * 1.4426950408889634f;  // scores to log2 units
+    float m_used = -INFINITY, l_part = 0.f;
 
-      // exchange the split-K halves of the score tile with the peer CTA
-      if (j >= 2) wait_cluster(smem_u32(&bars->x_free[u]), ((j >> 1) - 1) & 1, ab);
+    // This CTA's half of the query: 256 latent bf16 into TMEM (warp half 0
+    // columns 0..127, half 1 columns 128..255), 32 rotary bf16 into shared
+    // memory as a 64B-swizzled K-major row (warp half 1).
+    {
+      const uint4* ql = reinterpret_cast<const uint4*>(q_lat + ((size_t)b * kH + i) * kDl + rank * 256);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint32_t a = x_peer[u] + (uint32_t)((q * kH + i) * 16);
-        asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(sv[4 * q]),
-                     "r"(sv[4 * q + 1]), "r"(sv[4 * q + 2]), "r"(sv[4 * q + 3])
-                     : "memory");
+      for (int pp = 0; pp < 2; ++pp) {  // 64 latent values = 32 columns each
+        const int part = 2 * hf + pp;
+        uint32_t r[32];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const uint4 x = __ldg(ql + part * 8 + v);
+          r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
+        }
+        tmem_st32(tmem + lane_base + kColQ + part * 32, r);
       }
-      mbar_arrive_remote(xfull_peer[u]);
-      wait_cluster(smem_u32(&bars->x_full[u]), (j >> 1) & 1, ab);
+      if (hf == 1) {
+        const uint4* qp = reinterpret_cast<const uint4*>(q_pe + ((size_t)b * kH + i) * kDr + rank * 32);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 x = __ldg(qp + v);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sQpe + sw64_offset(i, v)), "r"(x.x),
+                       "r"(x.y), "r"(x.z), "r"(x.w)
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));
+    }
+
+    for (int j = 0; j < n_tiles; ++j) {
+      const uint32_t sbuf = tmem + lane_base + kColS + (j & 1) * kNt;
+      // full scores of tile j (this warp's 32 positions)
+      uint32_t sv[32];
+      wait(smem_u32(&bars->s_sum[j & 1]), (j >> 1) & 1, ab);
+      tc_fence_after();
+      if (leader) MLA_TRACE_STAMP(kTrSmStart, j);
+      tmem_ld32(sbuf + 32 * hf, sv);
+      // valid positions of tile j, published by the gather warp with the
+      // tile (the stage cannot be refilled before P(j) is written)
+      const int st = j % kStages;
+      wait(smem_u32(&bars->kv_full[st]), (j / kStages) & 1, ab);
+      const uint32_t vmask = *reinterpret_cast<volatile uint32_t*>(&bars->vmask[st][hf]);
+      tmem_wait_ld();
+
       float s[32];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float4 o = *reinterpret_cast<const float4*>(smem + kOffX + u * kXBytes + (q * kH + i) * 16);
-        s[4 * q + 0] = __uint_as_float(sv[4 * q + 0]) + o.x;
-        s[4 * q + 1] = __uint_as_float(sv[4 * q + 1]) + o.y;
-        s[4 * q + 2] = __uint_as_float(sv[4 * q + 2]) + o.z;
-        s[4 * q + 3] = __uint_as_float(sv[4 * q + 3]) + o.w;
-      }
-      mbar_arrive_remote(xfree_peer[u]);
-
-      // online softmax in log2 units
       float mx = -INFINITY;
 #pragma unroll
       for (int t = 0; t < 32; ++t) {
-        s[t] = ((vmask >> t) & 1u) ? s[t] * c2 : -INFINITY;
+        s[t] = ((vmask >> t) & 1u) ? __uint_as_float(sv[t]) * c2 : -INFINITY;  // log2 units; masked -> -inf
         mx = fmaxf(mx, s[t]);
       }
+      // the row maximum over all 64 positions, shared with the partner warp
+      // (after this barrier both warps of the pair have read their scores,
+      // so P may be written over them)
+      red[((j & 1) * 2 + hf) * kH + i] = mx;
+      named_bar_sync(1 + qd, 64);
+      mx = fmaxf(mx, red[((j & 1) * 2 + (hf ^ 1)) * kH + i]);
+      if (leader) MLA_TRACE_STAMP(kTrMaxShared, j);
+
       // The running maximum of a row moves only when the tile's maximum
       // exceeds it by more than 2^8 (so p <= 256 otherwise).  The TMEM
       // accesses are warp-collective, so the whole warp rescales when any of
-      // its rows must; rows that keep their maximum use alpha = 1.
+      // its rows must (both warps of a pair decide alike); rows that keep
+      // their maximum use alpha = 1.  Each warp of the pair rescales half of
+      // the row.
       const bool grow = mx > m_used + kRescaleThreshold;
       const float alpha = grow ? ((m_used == -INFINITY) ? 0.f : ex2_approx(m_used - mx)) : 1.f;
       if (__any_sync(0xffffffffu, grow) && j > 0) {
-        // PV(j-1) must have finished before O is rescaled in place
-        wait(smem_u32(&bars->o_done), (j - 1) & 1, ab);
+        // PV(j-1) (and so every earlier MMA) must have finished before O is
+        // rescaled in place
+        wait(smem_u32(&bars->p_free[(j - 1) & 1]), ((j - 1) >> 1) & 1, ab);
         tc_fence_after();
 #pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
+        for (int cc = 0; cc < 4; ++cc) {
+          const uint32_t col = kColO + 128 * hf + cc * 32;
           uint32_t ov[32];
-          tmem_ld32(tmem + lane_base + kColO + cc * 32, ov);
+          tmem_ld32(tmem + lane_base + col, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int t = 0; t < 32; ++t) ov[t] = __float_as_uint(__uint_as_float(ov[t]) * alpha);
-          tmem_st32(tmem + lane_base + kColO + cc * 32, ov);
+          tmem_st32(tmem + lane_base + col, ov);
         }
         tmem_wait_st();
       }
-      l_sum *= alpha;
+      l_part *= alpha;
       if (grow) m_used = mx;
+
+      // Masked positions hold -inf and give exp2(-inf) = 0.  While a row has
+      // seen no valid position its maximum is still -inf; subtracting 0 then
+      // keeps every masked term at exactly 0 instead of exp2(NaN).
+      const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
       uint32_t pk[16];
+      float lt = 0.f;
 #pragma unroll
       for (int t = 0; t < 16; ++t) {
-        const bool v0 = (vmask >> (2 * t)) & 1u, v1 = (vmask >> (2 * t + 1)) & 1u;
-        const float p0 = v0 ? ex2_approx(s[2 * t] - m_used) : 0.f;
-        const float p1 = v1 ? ex2_approx(s[2 * t + 1] - m_used) : 0.f;
+        const float p0 = ex2_approx(s[2 * t] - m_sub);
+        const float p1 = ex2_approx(s[2 * t + 1] - m_sub);
         pk[t] = pack_bf16x2(p0, p1);
-        const float2 r = unpack_bf16x2(pk[t]);  // the values the MMA will use
-        l_sum += r.x + r.y;
+        lt += p0 + p1;
       }
-      tmem_st16(tmem + lane_base + kColP + u * (kNt / 2), pk);
+      l_part += lt;
+      // P(j) over the first kNt/2 columns of the buffer; this warp's 32
+      // positions are columns [16hf, 16hf+16)
+      tmem_st16(sbuf + 16 * hf, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&bars->p_full[u]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[j & 1]));
+      if (leader) MLA_TRACE_STAMP(kTrPWritten, j);
     }
 
-    // epilogue: normalised O half and log-sum-exp of this split
-    float* orow = o_part + (((size_t)b * n_split + split) * kH + i) * kDl + rank * 256;
+    // epilogue: row sums of the pair combined, normalised O half and the
+    // split's log-sum-exp
+    red[((n_tiles & 1) * 2 + hf) * kH + i] = l_part;  // buffer not used by the last tile
+    named_bar_sync(1 + qd, 64);
+    const float l_sum = l_part + red[((n_tiles & 1) * 2 + (hf ^ 1)) * kH + i];
+    float* orow = o_part + (((size_t)b * n_split + split) * kH + i) * kDl + rank * 256 + 128 * hf;
     if (n_tiles > 0) {
-      wait(smem_u32(&bars->o_done), (n_tiles - 1) & 1, ab);
+      // the last PV done implies every MMA of the split is done
+      wait(smem_u32(&bars->p_free[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, ab);
       tc_fence_after();
     }
     const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
 #pragma unroll 1
-    for (int cc = 0; cc < 8; ++cc) {
+    for (int cc = 0; cc < 4; ++cc) {
       uint32_t ov[32];
       if (n_tiles > 0) {
-        tmem_ld32(tmem + lane_base + kColO + cc * 32, ov);
+        tmem_ld32(tmem + lane_base + kColO + 128 * hf + cc * 32, ov);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -469,7 +640,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
         *reinterpret_cast<float4*>(orow + cc * 32 + t) = v;
       }
     }
-    if (rank == 0) {
+    if (rank == 0 && hf == 0) {
       lse_part[((size_t)b * n_split + split) * kH + i] =
           l_sum > 0.f ? (m_used + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
     }
@@ -480,7 +651,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 4) tmem_dealloc(tmem, 512);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
   cluster_sync();
 }
 

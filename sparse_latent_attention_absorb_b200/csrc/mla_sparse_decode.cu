@@ -297,3 +297,13 @@ extern "C" int mla_sparse_decode(const void* q_nope, const void* q_pe, const voi
     return rc;
   return launch_combine(o_part, lse_part, wkv_b, out, lse_out, B, n_split, d_status, stream);
 }
+
+#ifdef MLA_TRACE
+// Trace builds only: copies the pipeline trace of the last traced launch
+// (2 CTAs x kTrEvents x kTraceTiles clock64 stamps) to host memory.
+extern "C" int mla_trace_fetch(long long* host, int n) {
+  const int total = 2 * kTrEvents * kTraceTiles;
+  if (!host || n < total) return MLA_ERR_INVALID_ARG;
+  return cudaMemcpyFromSymbol(host, g_mla_trace, sizeof(long long) * total) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+#endif

@@ -78,6 +78,11 @@ SMALL_WORKLOADS = {
     "small_b2_ctx9000_runs6x37": Workload(
         "small_b2_ctx9000_runs6x37", 2, 9000, (9000, 9000), 222, "runs", 2005, run_len=37, n_runs=6),
     "small_b2_ctx500_dense": Workload("small_b2_ctx500_dense", 2, 500, (500, 500), 500, "dense", 2006),
+    # enough rows that every row is one split of many tiles (online softmax
+    # across tiles, the gather ring wrapping around, double-buffered P)
+    "small_b80_ctx700_top300": Workload("small_b80_ctx700_top300", 80, 700, (700, 700), 300, "uniform", 2007),
+    "small_b76_ctx150-2k_recent64_top700": Workload(
+        "small_b76_ctx150-2k_recent64_top700", 76, 2048, (150, 2048), 700, "recent", 2008, recent=64),
 }
 
 ALL_WORKLOADS = {**WORKLOADS, **SMALL_WORKLOADS}
