@@ -135,6 +135,40 @@ int mla_sparse_attend(const void* q_lat, const void* q_pe, const void* kv_cache,
 int mla_combine_value_up(const float* o_part, const float* lse_part, const void* wkv_b, void* out,
                          float* lse_out, int B, int n_split, cudaStream_t stream);
 
+/*
+ * Size of the library's fixed device scratch used by
+ * mla_sparse_decode_noalloc (32 MiB, enough for B = 64 rows with K = 2048 on
+ * a 148-SM device; mla_sparse_decode_workspace_size() tells the need).
+ */
+#define MLA_STATIC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * The whole decode step without a workspace argument.  The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory when they call -- for example a plugin whose host framework
+ * owns all device memory and offers it no allocation hook, or a serving loop
+ * that must not call cudaMalloc, which can block and synchronise the device.
+ * It allocates nothing: the scratch is a fixed device array of
+ * MLA_STATIC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits.
+ *   - Arguments, layouts and results are those of mla_sparse_decode minus the
+ *     workspace.
+ *   - Sizes whose mla_sparse_decode_workspace_size() exceeds
+ *     MLA_STATIC_SCRATCH_BYTES are rejected with MLA_ERR_WORKSPACE before
+ *     anything is launched.
+ *   - The first call on a device looks up the array's device address (a
+ *     host-side CUDA runtime call, made with that device current); make that
+ *     first call before any stream capture.
+ *   - Every call shares the one array, and it keeps whatever the last call
+ *     left there (nothing in it needs to start at zero): calls whose work
+ *     overlaps on the GPU (different streams, or different host threads)
+ *     race on it.  Serialise them, e.g. on one stream.
+ */
+int mla_sparse_decode_noalloc(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                              const int32_t* end_pos, const int32_t* topk_idx, const void* wkv_b, float scale,
+                              void* out, int B, int K, int S_max, float* lse_out, int* d_status,
+                              cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

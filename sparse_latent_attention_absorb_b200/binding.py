@@ -22,7 +22,8 @@ STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_WORKSPACE", 3: "MLA
 
 # Every symbol the public header declares.
 EXPORTS = ("mla_status_string", "mla_num_splits", "mla_sparse_decode_workspace_size", "mla_sparse_decode",
-           "mla_absorb_q", "mla_sparse_attend", "mla_combine_value_up")
+           "mla_absorb_q", "mla_sparse_attend", "mla_combine_value_up", "mla_sparse_decode_noalloc")
+STATIC_SCRATCH_BYTES = 32 << 20  # MLA_STATIC_SCRATCH_BYTES
 
 _lib = None
 
@@ -56,6 +57,8 @@ def load_library():
     lib.mla_sparse_attend.argtypes = [p, p, p, p, p, p, f, p, p, i, i, i, i, p, p]
     lib.mla_combine_value_up.restype = i
     lib.mla_combine_value_up.argtypes = [p, p, p, p, p, i, i, p]
+    lib.mla_sparse_decode_noalloc.restype = i
+    lib.mla_sparse_decode_noalloc.argtypes = [p, p, p, p, p, p, p, f, p, i, i, i, p, p, p]
     _lib = lib
     return lib
 

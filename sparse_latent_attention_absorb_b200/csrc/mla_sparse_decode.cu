@@ -196,6 +196,27 @@ int prepare(DeviceInfo** info) {
   return get_encoder();
 }
 
+// Fixed device scratch for mla_sparse_decode_noalloc: one array per device
+// that loads the library, alive until the process exits.  Host code only sees
+// a stand-in for it, so its device address is looked up once per device.
+__device__ __align__(256) uint8_t g_mla_static_scratch[MLA_STATIC_SCRATCH_BYTES];
+void* g_static_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_mla_static_scratch on the current device (resolved on
+// the first call made with that device current).
+int static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_static_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_mla_static_scratch) != cudaSuccess || p == nullptr) return MLA_ERR_CUDA;
+    g_static_scratch_addr[dev] = p;
+  }
+  *out = g_static_scratch_addr[dev];
+  return MLA_OK;
+}
+
 }  // namespace
 
 // =============================================================================
@@ -307,3 +328,28 @@ extern "C" int mla_trace_fetch(long long* host, int n) {
   return cudaMemcpyFromSymbol(host, g_mla_trace, sizeof(long long) * total) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 #endif
+
+// The decode step without a caller-provided workspace: the scratch lives in
+// the library's fixed device array (see the header for who needs this).
+// Everything it holds is written before it is read, so nothing is cleared.
+extern "C" int mla_sparse_decode_noalloc(const void* q_nope, const void* q_pe, const void* kv_cache,
+                                         const void* pe_cache, const int32_t* end_pos, const int32_t* topk_idx,
+                                         const void* wkv_b, float scale, void* out, int B, int K, int S_max,
+                                         float* lse_out, int* d_status, cudaStream_t stream) {
+  const void* ptrs[] = {q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, out};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  if (lse_out && (reinterpret_cast<uintptr_t>(lse_out) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (!sizes_ok(B, K, S_max) || !std::isfinite(scale)) return MLA_ERR_INVALID_ARG;
+  DeviceInfo* info = nullptr;
+  int rc = prepare(&info);
+  if (rc != MLA_OK) return rc;
+  int n_split = 0, span = 0;
+  plan_splits(B, K, info->sm_count, &n_split, &span);
+  if (workspace_layout(B, n_split).total > (size_t)MLA_STATIC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((rc = static_scratch_address(&scratch)) != MLA_OK) return rc;
+  return mla_sparse_decode(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, scale, out, B, K, S_max,
+                           scratch, (size_t)MLA_STATIC_SCRATCH_BYTES, lse_out, d_status, stream);
+}
