@@ -134,9 +134,10 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 //
 // One 2-CTA cluster per (batch row b, key split s).  CTA rank r owns latent
 // columns [256r, 256r+256) and rotary columns [32r, 32r+32) of the score:
-//   * its half of the absorbed query is an MMA operand: q_lat[b, :, its 256]
-//     in TMEM (bf16 pairs), q_pe[b, :, its 32] in shared memory;
-//   * for every selected position t of the split, four gather warps copy
+//   * its half of the absorbed query is the A operand of QK: latent columns
+//     0..127 of the half in TMEM (bf16 pairs), columns 128..255 and the
+//     rotary part in shared memory;
+//   * for every selected position t of the split, three gather warps copy
 //     kv[b,t,its 256] (128B-swizzled rows) and pe[b,t,its 32] (64B-swizzled
 //     rows) into a ring of 64-position tiles (cp.async, 16 bytes per lane);
 //     padding positions are zero-filled without a read;
@@ -144,35 +145,39 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 //     pe[t, its 32]  -- a split-K half of the 576-wide score, M = 128 heads,
 //     N = 64 positions, into a TMEM score buffer;
 //   * four exchange warps swap the halves through distributed shared memory
-//     (st.async with transaction counts on the receiver's mbarrier) and write
-//     the full score S = S_0 + S_1 back into the buffer (bitwise identical in
-//     both CTAs: fp32 addition commutes), one tile ahead of the softmax;
-//   * eight softmax warps: online softmax with a lazily updated running
-//     maximum (O is rescaled only when the maximum grows by more than 2^8);
-//     P (bf16) is written into the same TMEM buffer over the scores;
+//     (st.async with transaction counts on the receiver's mbarrier), form the
+//     full score S = S_0 + S_1 (bitwise identical in both CTAs: fp32 addition
+//     commutes), mask and scale it to log2 units, write it back and publish
+//     each row's maximum over the tile;
+//   * eight softmax warps read the scores (which frees the buffer for the QK
+//     two tiles ahead), update the running maximum lazily (O is rescaled only
+//     when a row maximum grows by more than 2^8) and write P (bf16) into its
+//     own TMEM buffer;
 //   * PV: O_r[h, its 256] += P[h,t] . kv[t, its 256]  (A = P from TMEM,
-//     B = the same gathered rows read M/N-major).  tcgen05.mma operations of
-//     one CTA execute in issue order, so QK(j+2) issued after PV(j) may
-//     overwrite the buffer that holds P(j).
+//     B = the same gathered rows read M/N-major).
 // The split's normalised O and its log-sum-exp go to o_part / lse_part.
 //
-// Warp roles (544 threads): warps 0-7 softmax (warps w and w+4 share TMEM
+// Warp roles (512 threads): warps 0-7 softmax (warps w and w+4 share TMEM
 // lanes 32(w%4).. and take positions 0-31 / 32-63 of every tile); warps 8-11
 // score exchange (lanes 32(w%4).., all 64 positions); warp 12 TMEM
-// allocation + MMA issue; warps 13-16 gather (one stage each).
+// allocation + MMA issue; warps 13-15 gather (one stage each).
 // =============================================================================
 constexpr int kNt = 64;                            // positions per tile
-constexpr int kStages = 4;                         // gathered tile ring
+constexpr int kStages = 3;                         // gathered tile ring
 constexpr int kXBufs = 2;                          // score-exchange buffers
 constexpr int kLatBlock = kNt * 128;               // one 64-column latent block of a tile (8 KB)
 constexpr int kStageBytes = 4 * kLatBlock + kNt * 64;  // 4 latent blocks + the rotary block: 36 KB
+constexpr int kQsBytes = 2 * kH * 128;             // latent query columns 128..255 of the half: 32 KB
 constexpr int kQpeBytes = kH * 64;                 // 8 KB
 constexpr int kXBytes = (kNt / 4) * kH * 16;       // 32 KB: one exchanged score tile (f32)
-constexpr int kRedBytes = 2 * 2 * kH * 4;          // row maxima / sums shared by warp pairs
+constexpr int kTmaxBytes = 2 * kH * 4;             // tile row maxima, by tile parity
+constexpr int kRedBytes = 2 * kH * 4;              // row sums of the warp pairs at the end
 constexpr int kOffStage = 0;
 constexpr int kOffX = kOffStage + kStages * kStageBytes;
-constexpr int kOffQpe = kOffX + kXBufs * kXBytes;
-constexpr int kOffRed = kOffQpe + kQpeBytes;
+constexpr int kOffQs = kOffX + kXBufs * kXBytes;
+constexpr int kOffQpe = kOffQs + kQsBytes;
+constexpr int kOffTmax = kOffQpe + kQpeBytes;
+constexpr int kOffRed = kOffTmax + kTmaxBytes;
 constexpr int kOffBar = kOffRed + kRedBytes;
 constexpr int kAttendSmemBytes = kOffBar + 256 + kSmemAlignPad;
 constexpr int kSoftmaxWarps = 8;
@@ -181,16 +186,18 @@ constexpr int kXchgWarps = 4;
 constexpr int kMmaWarp = 12;
 constexpr int kGatherWarp0 = 13;
 constexpr int kGatherWarps = kStages;  // gather warp g always fills stage g
-constexpr int kAttendThreads = 32 * (kGatherWarp0 + kGatherWarps);  // 544
+constexpr int kAttendThreads = 32 * (kGatherWarp0 + kGatherWarps);  // 512
 // TMEM columns
-constexpr uint32_t kColS = 0;     // two score buffers of kNt f32 columns; P (bf16 pairs) over the first kNt/2
-constexpr uint32_t kColQ = 128;   // 128 columns: 256 bf16 of the latent query half
+constexpr uint32_t kColS = 0;     // two score buffers of kNt f32 columns
+constexpr uint32_t kColP = 128;   // two P buffers of kNt/2 columns (bf16 pairs)
+constexpr uint32_t kColQ = 192;   // 64 columns: latent query columns 0..127 of the half (bf16 pairs)
 constexpr uint32_t kColO = 256;   // 256 f32 columns of O
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-static_assert(kStageBytes % 1024 == 0 && kOffX % 1024 == 0 && kOffQpe % 1024 == 0, "swizzle atoms");
+static_assert(kStageBytes % 1024 == 0 && kOffX % 1024 == 0 && kOffQs % 1024 == 0 && kOffQpe % 1024 == 0,
+              "swizzle atoms");
 static_assert(kAttendSmemBytes <= 232448, "shared memory");
-static_assert(kColS + 2 * kNt <= kColQ && kColQ + 128 <= kColO, "TMEM map");
+static_assert(kColS + 2 * kNt <= kColP && kColP + kNt <= kColQ && kColQ + 64 <= kColO, "TMEM map");
 // Exchange buffers: the exchange warps of a CTA push tile t into the peer's
 // buffer t mod 2 after they have received the peer's push of tile t-1, which
 // every peer exchange warp issued after it had read tile t-2 from that same
@@ -208,9 +215,10 @@ struct AttendBars {
   uint64_t kv_full[kStages];    // the tile's gather warp (1 arrival) once its copies landed
   uint64_t kv_empty[kStages];   // MMA commit after PV of the tile
   uint64_t s_full[2];           // MMA commit after QK: partial scores in the buffer
-  uint64_t s_sum[2];            // exchange warps (4) after writing the full scores back
-  uint64_t p_full[2];           // softmax warps (8) after writing P over the scores
-  uint64_t p_free[2];           // MMA commit after PV of the tile: O stable
+  uint64_t s_sum[2];            // exchange warps (4): scaled full scores and tile maxima ready
+  uint64_t s_empty[2];          // softmax warps (8) after reading the scores
+  uint64_t p_full[2];           // softmax warps (8) after writing P
+  uint64_t p_free[2];           // MMA commit after PV of the tile: P buffer free, O stable
   uint64_t x_full[kXBufs];      // 1 local arrival + kXBytes from the peer's st.async
   uint32_t vmask[kStages][2];   // valid positions of the tile in each stage (bit n of word n/32)
   uint32_t tmem_addr;
@@ -237,9 +245,9 @@ enum TraceEvent {
   kTrXStart,           // exchange warp 8: partial scores of the tile available
   kTrXPushed,          // exchange warp 8: partial scores pushed to the peer
   kTrXArrived,         // exchange warp 8: peer's partial scores observed
-  kTrXSummed,          // exchange warp 8: full scores written back
-  kTrSmStart,          // softmax warp 0: full scores of the tile available
-  kTrMaxShared,        // softmax warp 0: tile maximum shared with its partner warp
+  kTrXSummed,          // exchange warp 8: scaled full scores written back
+  kTrSmStart,          // softmax warp 0: scores of the tile available
+  kTrSmRead,           // softmax warp 0: scores read, buffer released
   kTrPWritten,         // softmax warp 0: P of the tile written, p_full arrived
   kTrEvents
 };
@@ -280,10 +288,13 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
 
   const uint32_t sStage = smem_u32(smem + kOffStage);
   const uint32_t sX = smem_u32(smem + kOffX);
+  const uint32_t sQs = smem_u32(smem + kOffQs);
   const uint32_t sQpe = smem_u32(smem + kOffQpe);
-  float* red = reinterpret_cast<float*>(smem + kOffRed);  // [tile parity][half][head]
+  float* tmax = reinterpret_cast<float*>(smem + kOffTmax);  // [tile parity][head]
+  float* red = reinterpret_cast<float*>(smem + kOffRed);    // [half][head]
   AttendBars* bars = reinterpret_cast<AttendBars*>(smem + kOffBar);
   const AbortState ab{&bars->abort_flag, d_status};
+  const float c2 = scale * 1.4426950408889634f;  // scores to log2 units
 
   if (tid == 0) {
     bars->abort_flag = 0;
@@ -295,6 +306,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars->s_full[i]), 1);
       mbar_init(smem_u32(&bars->s_sum[i]), kXchgWarps);
+      mbar_init(smem_u32(&bars->s_empty[i]), kSoftmaxWarps);
       mbar_init(smem_u32(&bars->p_full[i]), kSoftmaxWarps);
       mbar_init(smem_u32(&bars->p_free[i]), 1);
     }
@@ -315,7 +327,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
 
   if (warp >= kGatherWarp0) {
     // ------------------------------------------------------------ gather
-    // Gather warp g owns stage g and tiles g, g+4, g+8, ...; lane l handles
+    // Gather warp g owns stage g and tiles g, g+3, g+6, ...; lane l handles
     // positions l and l+32 of a tile.  Latent: one position per instruction
     // (32 lanes x 16 bytes = this CTA's 256 columns); rotary: eight positions
     // per instruction (this CTA's 32 columns).  A tile is published
@@ -366,23 +378,38 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     };
     // this warp's next two tiles, statically indexed (a register copy of a
     // pending load would wait for the load)
+    // Rows of this warp's next tile are pulled into L2 while the tile ahead
+    // of it is still in use, so its copies hit L2 once the stage frees.
+    auto prefetch_tile = [&](int idx0, int idx1) {
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int pos = h2 ? idx1 : idx0;
+        if (pos >= 0) {
+          const char* r = reinterpret_cast<const char*>(kv_row0 + (size_t)pos * kDl);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) asm volatile("prefetch.global.L2 [%0];" ::"l"(r + c * 128));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(pe_row0 + (size_t)pos * kDr));
+        }
+      }
+    };
     int a0 = load_idx(g, 0), a1 = load_idx(g, 1);
     int b0 = load_idx(g + kStages, 0), b1 = load_idx(g + kStages, 1);
     for (int j = g; j < n_tiles; j += 2 * kStages) {
       gather_tile(j, a0, a1);
+      prefetch_tile(b0, b1);
       a0 = load_idx(j + 2 * kStages, 0);
       a1 = load_idx(j + 2 * kStages, 1);
       if (j + kStages < n_tiles) {
         gather_tile(j + kStages, b0, b1);
+        prefetch_tile(a0, a1);
         b0 = load_idx(j + 3 * kStages, 0);
         b1 = load_idx(j + 3 * kStages, 1);
       }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
-    // In order: QK(0), QK(1), then for every tile j: PV(j) once P(j) is
-    // written, then QK(j+2) into the buffer P(j) occupied once its rows have
-    // landed.
+    // A polling scheduler: PV(pv) as soon as P is written, QK(qk) as soon as
+    // its rows have landed and its score buffer has been read, PV first.
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kNt, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
@@ -390,44 +417,70 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       // is the base descriptor plus x/16 (start-address field).
       const uint64_t d_lat = smem_desc_sw128(sStage, 16, 1024);            // QK B, latent, K-major
       const uint64_t d_pe = smem_desc_sw64(sStage + 4 * kLatBlock, 512);    // QK B, rotary, K-major
+      const uint64_t d_qs = smem_desc_sw128(sQs, 16, 1024);                 // QK A, latent 128..255, K-major
       const uint64_t d_qpe = smem_desc_sw64(sQpe, 512);                     // QK A, rotary, K-major
       const uint64_t d_v = smem_desc_sw128(sStage, kLatBlock, 1024);        // PV B, latent, N-major
       wait(smem_u32(&bars->q_full), 0, ab);
       tc_fence_after();
-      auto issue_qk = [&](int t) {
-        const int st = t % kStages;
-        wait(smem_u32(&bars->kv_full[st]), (t / kStages) & 1, ab);
-        tc_fence_after();
-        MLA_TRACE_STAMP(kTrQkStart, t);
-        const uint64_t dl = d_lat + (uint64_t)((st * kStageBytes) >> 4);
-        const uint64_t dr = d_pe + (uint64_t)((st * kStageBytes) >> 4);
-        const uint32_t dst = tmem + kColS + (t & 1) * kNt;
+      int qk = 0, pv = 0, st_qk = 0, st_pv = 0;
+      uint32_t idle = 0;
+      uint64_t idle_since = 0;
+      while (pv < n_tiles) {
+        bool did = false;
+        if (pv < qk && mbar_test(smem_u32(&bars->p_full[pv & 1]), (pv >> 1) & 1)) {
+          tc_fence_after();
+          MLA_TRACE_STAMP(kTrPvStart, pv);
+          const uint64_t dv = d_v + (uint64_t)((st_pv * kStageBytes) >> 4);
+          const uint32_t pa = tmem + kColP + (pv & 1) * (kNt / 2);
 #pragma unroll
-        for (int k = 0; k < 16; ++k)  // latent: K block k/4, 32 bytes per step
-          mma_ts(dst, tmem + kColQ + k * 8, dl + (uint64_t)(((k >> 2) * kLatBlock + (k & 3) * 32) >> 4), idesc_qk,
-                 k > 0 ? 1u : 0u);
+          for (int k = 0; k < kNt / 16; ++k)  // 16 positions per step
+            mma_ts(tmem + kColO, pa + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4), idesc_pv,
+                   (pv > 0 || k > 0) ? 1u : 0u);
+          mma_commit(smem_u32(&bars->kv_empty[st_pv]));
+          mma_commit(smem_u32(&bars->p_free[pv & 1]));
+          MLA_TRACE_STAMP(kTrPvIssued, pv);
+          ++pv;
+          st_pv = (st_pv + 1 == kStages) ? 0 : st_pv + 1;
+          did = true;
+        } else if (qk < n_tiles && mbar_test(smem_u32(&bars->kv_full[st_qk]), (qk / kStages) & 1) &&
+                   (qk < 2 || mbar_test(smem_u32(&bars->s_empty[qk & 1]), ((qk >> 1) - 1) & 1))) {
+          tc_fence_after();
+          MLA_TRACE_STAMP(kTrQkStart, qk);
+          const uint64_t dl = d_lat + (uint64_t)((st_qk * kStageBytes) >> 4);
+          const uint64_t dr = d_pe + (uint64_t)((st_qk * kStageBytes) >> 4);
+          const uint32_t dst = tmem + kColS + (qk & 1) * kNt;
 #pragma unroll
-        for (int k = 0; k < 2; ++k)  // rotary: 32 bytes per step inside the 64-byte rows
-          mma_ss(dst, d_qpe + (uint64_t)((k * 32) >> 4), dr + (uint64_t)((k * 32) >> 4), idesc_qk, 1u);
-        mma_commit(smem_u32(&bars->s_full[t & 1]));
-        MLA_TRACE_STAMP(kTrQkIssued, t);
-      };
-      issue_qk(0);
-      if (n_tiles > 1) issue_qk(1);
-      for (int j = 0; j < n_tiles; ++j) {
-        const int st = j % kStages;
-        wait(smem_u32(&bars->p_full[j & 1]), (j >> 1) & 1, ab);
-        tc_fence_after();
-        MLA_TRACE_STAMP(kTrPvStart, j);
-        const uint64_t dv = d_v + (uint64_t)((st * kStageBytes) >> 4);
-        const uint32_t pa = tmem + kColS + (j & 1) * kNt;  // P(j): kNt/2 columns of bf16 pairs
+          for (int k = 0; k < 8; ++k)  // latent 0..127: A from TMEM
+            mma_ts(dst, tmem + kColQ + k * 8, dl + (uint64_t)(((k >> 2) * kLatBlock + (k & 3) * 32) >> 4), idesc_qk,
+                   k > 0 ? 1u : 0u);
 #pragma unroll
-        for (int k = 0; k < kNt / 16; ++k)  // 16 positions per step
-          mma_ts(tmem + kColO, pa + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
-        mma_commit(smem_u32(&bars->kv_empty[st]));
-        mma_commit(smem_u32(&bars->p_free[j & 1]));
-        MLA_TRACE_STAMP(kTrPvIssued, j);
-        if (j + 2 < n_tiles) issue_qk(j + 2);
+          for (int k = 8; k < 16; ++k)  // latent 128..255: A from shared memory
+            mma_ss(dst, d_qs + (uint64_t)((((k - 8) >> 2) * (kH * 128) + (k & 3) * 32) >> 4),
+                   dl + (uint64_t)(((k >> 2) * kLatBlock + (k & 3) * 32) >> 4), idesc_qk, 1u);
+#pragma unroll
+          for (int k = 0; k < 2; ++k)  // rotary: 32 bytes per step inside the 64-byte rows
+            mma_ss(dst, d_qpe + (uint64_t)((k * 32) >> 4), dr + (uint64_t)((k * 32) >> 4), idesc_qk, 1u);
+          mma_commit(smem_u32(&bars->s_full[qk & 1]));
+          MLA_TRACE_STAMP(kTrQkIssued, qk);
+          ++qk;
+          st_qk = (st_qk + 1 == kStages) ? 0 : st_qk + 1;
+          did = true;
+        }
+        if (did) {
+          idle = 0;
+        } else if (idle++ == 0) {
+          idle_since = global_timer_ns();
+        } else {
+          __nanosleep(40);  // keep the barrier probes from crowding the shared-memory pipe
+        }
+        if (!did && (idle & 255u) == 0 && idle > 0) {
+          if (bars->abort_flag) break;
+          if (global_timer_ns() - idle_since > kWaitLimitNs) {
+            bars->abort_flag = 1;
+            if (d_status) atomicCAS(d_status, 0, MLA_ERR_DEVICE_TIMEOUT);
+            break;
+          }
+        }
       }
     }
     __syncwarp();
@@ -449,37 +502,42 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       wait(smem_u32(&bars->s_full[j & 1]), (j >> 1) & 1, ab);
       tc_fence_after();
       if (leader) MLA_TRACE_STAMP(kTrXStart, j);
+      uint32_t sv[64];
+      tmem_ld32(sbuf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(sbuf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_wait_ld();
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {  // positions [32 h2, 32 h2 + 32)
-        uint32_t sv[32];
-        tmem_ld32(sbuf + 32 * h2, sv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          st_async_v4(x_peer[u] + (uint32_t)(((8 * h2 + q) * kH + i) * 16), sv[4 * q], sv[4 * q + 1],
-                      sv[4 * q + 2], sv[4 * q + 3], xfull_peer[u]);
-      }
+      for (int q = 0; q < 16; ++q)
+        st_async_v4(x_peer[u] + (uint32_t)((q * kH + i) * 16), sv[4 * q], sv[4 * q + 1], sv[4 * q + 2],
+                    sv[4 * q + 3], xfull_peer[u]);
       if (leader) MLA_TRACE_STAMP(kTrXPushed, j);
+      // valid positions of tile j (the stage cannot be refilled before PV(j))
+      const int st = j % kStages;
+      wait(smem_u32(&bars->kv_full[st]), (j / kStages) & 1, ab);
+      const uint32_t vm0 = *reinterpret_cast<volatile uint32_t*>(&bars->vmask[st][0]);
+      const uint32_t vm1 = *reinterpret_cast<volatile uint32_t*>(&bars->vmask[st][1]);
       wait(smem_u32(&bars->x_full[u]), (j / kXBufs) & 1, ab);
       if (leader) {
         MLA_TRACE_STAMP(kTrXArrived, j);
         mbar_arrive_expect_tx(smem_u32(&bars->x_full[u]), kXBytes);  // re-arm for tile j + kXBufs
       }
+      float mx = -INFINITY;
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t sv[32];
-        tmem_ld32(sbuf + 32 * h2, sv);
-        tmem_wait_ld();
+      for (int q = 0; q < 16; ++q) {
+        const float4 o = *reinterpret_cast<const float4*>(smem + kOffX + u * kXBytes + (q * kH + i) * 16);
+        const float po[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 o = *reinterpret_cast<const float4*>(smem + kOffX + u * kXBytes + ((8 * h2 + q) * kH + i) * 16);
-          sv[4 * q + 0] = __float_as_uint(__uint_as_float(sv[4 * q + 0]) + o.x);
-          sv[4 * q + 1] = __float_as_uint(__uint_as_float(sv[4 * q + 1]) + o.y);
-          sv[4 * q + 2] = __float_as_uint(__uint_as_float(sv[4 * q + 2]) + o.z);
-          sv[4 * q + 3] = __float_as_uint(__uint_as_float(sv[4 * q + 3]) + o.w);
+        for (int e = 0; e < 4; ++e) {
+          const int t = 4 * q + e;
+          const bool v = (((t < 32) ? vm0 : vm1) >> (t & 31)) & 1u;
+          const float x = v ? (__uint_as_float(sv[t]) + po[e]) * c2 : -INFINITY;  // log2 units; masked -> -inf
+          mx = fmaxf(mx, x);
+          sv[t] = __float_as_uint(x);
         }
-        tmem_st32(sbuf + 32 * h2, sv);
       }
+      tmax[(j & 1) * kH + i] = mx;
+      tmem_st32(sbuf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_st32(sbuf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -493,26 +551,39 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     const int i = qd * 32 + lane;   // head
     const bool leader = (warp == 0 && lane == 0);
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
-    const float c2 = scale * 1.4426950408889634f;  // scores to log2 units
     float m_used = -INFINITY, l_part = 0.f;
 
-    // This CTA's half of the query: 256 latent bf16 into TMEM (warp half 0
-    // columns 0..127, half 1 columns 128..255), 32 rotary bf16 into shared
-    // memory as a 64B-swizzled K-major row (warp half 1).
+    // This CTA's half of the query: latent columns 0..127 into TMEM (warp
+    // half 0), latent columns 128..255 into shared memory as two 128B-
+    // swizzled K-major blocks and the 32 rotary values as a 64B-swizzled
+    // K-major row (warp half 1).
     {
       const uint4* ql = reinterpret_cast<const uint4*>(q_lat + ((size_t)b * kH + i) * kDl + rank * 256);
+      if (hf == 0) {
 #pragma unroll
-      for (int pp = 0; pp < 2; ++pp) {  // 64 latent values = 32 columns each
-        const int part = 2 * hf + pp;
-        uint32_t r[32];
+        for (int part = 0; part < 2; ++part) {  // 64 latent values = 32 columns each
+          uint32_t r[32];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const uint4 x = __ldg(ql + part * 8 + v);
-          r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
+          for (int v = 0; v < 8; ++v) {
+            const uint4 x = __ldg(ql + part * 8 + v);
+            r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
+          }
+          tmem_st32(tmem + lane_base + kColQ + part * 32, r);
         }
-        tmem_st32(tmem + lane_base + kColQ + part * 32, r);
-      }
-      if (hf == 1) {
+        tmem_wait_st();
+        tc_fence_before();
+      } else {
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint4 x = __ldg(ql + (2 + part) * 8 + v);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sQs + part * (kH * 128) +
+                                                                          sw128_offset(i, v)),
+                         "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w)
+                         : "memory");
+          }
+        }
         const uint4* qp = reinterpret_cast<const uint4*>(q_pe + ((size_t)b * kH + i) * kDr + rank * 32);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -523,41 +594,24 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
         }
         fence_proxy_async_smem();
       }
-      tmem_wait_st();
-      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));
     }
 
     for (int j = 0; j < n_tiles; ++j) {
-      const uint32_t sbuf = tmem + lane_base + kColS + (j & 1) * kNt;
-      // full scores of tile j (this warp's 32 positions)
+      // scaled, masked scores of tile j (this warp's 32 positions) and the
+      // row maxima over all 64, from the exchange warps
       uint32_t sv[32];
       wait(smem_u32(&bars->s_sum[j & 1]), (j >> 1) & 1, ab);
       tc_fence_after();
       if (leader) MLA_TRACE_STAMP(kTrSmStart, j);
-      tmem_ld32(sbuf + 32 * hf, sv);
-      // valid positions of tile j, published by the gather warp with the
-      // tile (the stage cannot be refilled before P(j) is written)
-      const int st = j % kStages;
-      wait(smem_u32(&bars->kv_full[st]), (j / kStages) & 1, ab);
-      const uint32_t vmask = *reinterpret_cast<volatile uint32_t*>(&bars->vmask[st][hf]);
+      tmem_ld32(tmem + lane_base + kColS + (j & 1) * kNt + 32 * hf, sv);
+      const float mx = tmax[(j & 1) * kH + i];
       tmem_wait_ld();
-
-      float s[32];
-      float mx = -INFINITY;
-#pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        s[t] = ((vmask >> t) & 1u) ? __uint_as_float(sv[t]) * c2 : -INFINITY;  // log2 units; masked -> -inf
-        mx = fmaxf(mx, s[t]);
-      }
-      // the row maximum over all 64 positions, shared with the partner warp
-      // (after this barrier both warps of the pair have read their scores,
-      // so P may be written over them)
-      red[((j & 1) * 2 + hf) * kH + i] = mx;
-      named_bar_sync(1 + qd, 64);
-      mx = fmaxf(mx, red[((j & 1) * 2 + (hf ^ 1)) * kH + i]);
-      if (leader) MLA_TRACE_STAMP(kTrMaxShared, j);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[j & 1]));
+      if (leader) MLA_TRACE_STAMP(kTrSmRead, j);
 
       // The running maximum of a row moves only when the tile's maximum
       // exceeds it by more than 2^8 (so p <= 256 otherwise).  The TMEM
@@ -595,15 +649,16 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       float lt = 0.f;
 #pragma unroll
       for (int t = 0; t < 16; ++t) {
-        const float p0 = ex2_approx(s[2 * t] - m_sub);
-        const float p1 = ex2_approx(s[2 * t + 1] - m_sub);
+        const float p0 = ex2_approx(__uint_as_float(sv[2 * t]) - m_sub);
+        const float p1 = ex2_approx(__uint_as_float(sv[2 * t + 1]) - m_sub);
         pk[t] = pack_bf16x2(p0, p1);
         lt += p0 + p1;
       }
       l_part += lt;
-      // P(j) over the first kNt/2 columns of the buffer; this warp's 32
-      // positions are columns [16hf, 16hf+16)
-      tmem_st16(sbuf + 16 * hf, pk);
+      // P buffer j&1 was last read by PV(j-2)
+      if (j >= 2) wait(smem_u32(&bars->p_free[j & 1]), ((j >> 1) - 1) & 1, ab);
+      tc_fence_after();
+      tmem_st16(tmem + lane_base + kColP + (j & 1) * (kNt / 2) + 16 * hf, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -613,9 +668,9 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
 
     // epilogue: row sums of the pair combined, normalised O half and the
     // split's log-sum-exp
-    red[((n_tiles & 1) * 2 + hf) * kH + i] = l_part;  // buffer not used by the last tile
+    red[hf * kH + i] = l_part;
     named_bar_sync(1 + qd, 64);
-    const float l_sum = l_part + red[((n_tiles & 1) * 2 + (hf ^ 1)) * kH + i];
+    const float l_sum = l_part + red[(hf ^ 1) * kH + i];
     float* orow = o_part + (((size_t)b * n_split + split) * kH + i) * kDl + rank * 256 + 128 * hf;
     if (n_tiles > 0) {
       // the last PV done implies every MMA of the split is done
