@@ -11,7 +11,9 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
+#include <cstring>
 
 #include "ptx.cuh"
 
@@ -137,99 +139,112 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 //   * its half of the absorbed query is the A operand of QK: latent columns
 //     0..127 of the half in TMEM (bf16 pairs), columns 128..255 and the
 //     rotary part in shared memory;
-//   * for every selected position t of the split, three gather warps copy
+//   * for every selected position t of the split, a gather warp copies
 //     kv[b,t,its 256] (128B-swizzled rows) and pe[b,t,its 32] (64B-swizzled
 //     rows) into a ring of 64-position tiles (cp.async, 16 bytes per lane);
 //     padding positions are zero-filled without a read;
 //   * QK: S_r[h,t] = q_lat[h, its 256] . kv[t, its 256] + q_pe[h, its 32] .
 //     pe[t, its 32]  -- a split-K half of the 576-wide score, M = 128 heads,
 //     N = 64 positions, into a TMEM score buffer;
-//   * four exchange warps swap the halves through distributed shared memory
-//     (st.async with transaction counts on the receiver's mbarrier), form the
-//     full score S = S_0 + S_1 (bitwise identical in both CTAs: fp32 addition
-//     commutes), mask and scale it to log2 units, write it back and publish
-//     each row's maximum over the tile;
-//   * eight softmax warps read the scores (which frees the buffer for the QK
-//     two tiles ahead), update the running maximum lazily (O is rescaled only
-//     when a row maximum grows by more than 2^8) and write P (bf16) into its
-//     own TMEM buffer;
+//   * two groups of four softmax warps take alternate tiles.  A thread owns
+//     one head (TMEM lane) and all 64 positions of its group's tiles: it
+//     reads its partial scores (which frees the buffer for the QK two tiles
+//     ahead), rounds them to fp16 in log2 units, pushes them into the peer
+//     CTA's shared memory (st.async, completing on the peer's mbarrier),
+//     adds the peer's half -- both CTAs add the same two fp16 values, so their
+//     scores and everything after are bitwise identical -- masks, takes the
+//     tile maximum, updates the running maximum lazily (O is rescaled only
+//     when a row maximum grows by more than 2^8; the groups hand the running
+//     maximum to each other tile by tile) and writes P (bf16) into its
+//     group's TMEM buffer;
 //   * PV: O_r[h, its 256] += P[h,t] . kv[t, its 256]  (A = P from TMEM,
 //     B = the same gathered rows read M/N-major).
 // The split's normalised O and its log-sum-exp go to o_part / lse_part.
 //
-// Warp roles (512 threads): warps 0-7 softmax (warps w and w+4 share TMEM
-// lanes 32(w%4).. and take positions 0-31 / 32-63 of every tile); warps 8-11
-// score exchange (lanes 32(w%4).., all 64 positions); warp 12 TMEM
-// allocation + MMA issue; warps 13-15 gather (one stage each).
+// Warp roles (416 threads): warps 0-3 softmax group 0 (even tiles), warps
+// 4-7 softmax group 1 (odd tiles), warp w covering TMEM lanes 32(w%4)..;
+// warp 8 TMEM allocation + MMA issue; warps 9-12 gather (one stage each).
 // =============================================================================
 constexpr int kNt = 64;                            // positions per tile
-constexpr int kStages = 3;                         // gathered tile ring
-constexpr int kXBufs = 2;                          // score-exchange buffers
+constexpr int kStages = 4;                         // gathered tile ring
 constexpr int kLatBlock = kNt * 128;               // one 64-column latent block of a tile (8 KB)
 constexpr int kStageBytes = 4 * kLatBlock + kNt * 64;  // 4 latent blocks + the rotary block: 36 KB
 constexpr int kQsBytes = 2 * kH * 128;             // latent query columns 128..255 of the half: 32 KB
 constexpr int kQpeBytes = kH * 64;                 // 8 KB
-constexpr int kXBytes = (kNt / 4) * kH * 16;       // 32 KB: one exchanged score tile (f32)
-constexpr int kTmaxBytes = 2 * kH * 4;             // tile row maxima, by tile parity
-constexpr int kRedBytes = 2 * kH * 4;              // row sums of the warp pairs at the end
+constexpr int kXHalves = (kNt / 8) * kH * 16;      // 16 KB: one exchanged score tile (fp16)
+constexpr int kXBytes = kXHalves + kH * 4;         // + each row's fp32 offset
+constexpr int kMslotBytes = 2 * kH * 4;            // running maximum published by each group
+constexpr int kRedBytes = 4 * kH * 4;              // (row sum, maximum) of each group at the end
+constexpr int kBarBytes = 512;
 constexpr int kOffStage = 0;
 constexpr int kOffX = kOffStage + kStages * kStageBytes;
-constexpr int kOffQs = kOffX + kXBufs * kXBytes;
+constexpr int kOffQs = kOffX + 2 * kXBytes;
 constexpr int kOffQpe = kOffQs + kQsBytes;
-constexpr int kOffTmax = kOffQpe + kQpeBytes;
-constexpr int kOffRed = kOffTmax + kTmaxBytes;
+constexpr int kOffMslot = kOffQpe + kQpeBytes;
+constexpr int kOffRed = kOffMslot + kMslotBytes;
 constexpr int kOffBar = kOffRed + kRedBytes;
-constexpr int kAttendSmemBytes = kOffBar + 256 + kSmemAlignPad;
-constexpr int kSoftmaxWarps = 8;
-constexpr int kXchgWarp0 = 8;
-constexpr int kXchgWarps = 4;
-constexpr int kMmaWarp = 12;
-constexpr int kGatherWarp0 = 13;
+constexpr int kAttendSmemBytes = kOffBar + kBarBytes + kSmemAlignPad;
+constexpr int kSoftmaxWarps = 8;                   // two groups of four
+constexpr int kMmaWarp = 8;
+constexpr int kGatherWarp0 = 9;
 constexpr int kGatherWarps = kStages;  // gather warp g always fills stage g
-constexpr int kAttendThreads = 32 * (kGatherWarp0 + kGatherWarps);  // 512
+// 13 warps: at most 128 registers a thread (the warps spread over the four
+// SM sub-partitions, 16K registers each, one of which holds four warps).
+constexpr int kAttendThreads = 32 * (kGatherWarp0 + kGatherWarps);  // 416
 // TMEM columns
-constexpr uint32_t kColS = 0;     // two score buffers of kNt f32 columns
-constexpr uint32_t kColP = 128;   // two P buffers of kNt/2 columns (bf16 pairs)
+constexpr uint32_t kColS = 0;     // score buffer of group g at kColS + 64g (f32)
+constexpr uint32_t kColP = 128;   // P buffer of group g at kColP + 32g (bf16 pairs)
 constexpr uint32_t kColQ = 192;   // 64 columns: latent query columns 0..127 of the half (bf16 pairs)
 constexpr uint32_t kColO = 256;   // 256 f32 columns of O
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-static_assert(kStageBytes % 1024 == 0 && kOffX % 1024 == 0 && kOffQs % 1024 == 0 && kOffQpe % 1024 == 0,
+static_assert(kStageBytes % 1024 == 0 && kOffX % 1024 == 0 && kOffQs % 1024 == 0 && kOffQpe % 1024 == 0 &&
+                  kXBytes % 16 == 0,
               "swizzle atoms");
 static_assert(kAttendSmemBytes <= 232448, "shared memory");
 static_assert(kColS + 2 * kNt <= kColP && kColP + kNt <= kColQ && kColQ + 64 <= kColO, "TMEM map");
-// Exchange buffers: the exchange warps of a CTA push tile t into the peer's
-// buffer t mod 2 after they have received the peer's push of tile t-1, which
-// every peer exchange warp issued after it had read tile t-2 from that same
-// buffer.
-static_assert(kXBufs >= 2, "score exchange reuse distance");
 // Each gather warp owns one stage (tiles g, g+kStages, ...), so every wait on
 // a stage's kv_empty barrier is exactly one phase after the warp's previous
 // wait on it; with fewer stages than warps a waiter could run two phases
 // ahead of the barrier, where a parity test cannot tell the phases apart.
 static_assert(kGatherWarps == kStages, "one stage per gather warp");
-static_assert(kXchgWarp0 % 4 == 0 && kXchgWarps == 4, "exchange warps cover the four TMEM lane quarters");
+static_assert(kMmaWarp == kSoftmaxWarps && kGatherWarp0 == kMmaWarp + 1, "warp roles");
 
 struct AttendBars {
   uint64_t q_full;              // softmax warps (8 arrivals) after storing Q
   uint64_t kv_full[kStages];    // the tile's gather warp (1 arrival) once its copies landed
   uint64_t kv_empty[kStages];   // MMA commit after PV of the tile
-  uint64_t s_full[2];           // MMA commit after QK: partial scores in the buffer
-  uint64_t s_sum[2];            // exchange warps (4): scaled full scores and tile maxima ready
-  uint64_t s_empty[2];          // softmax warps (8) after reading the scores
-  uint64_t p_full[2];           // softmax warps (8) after writing P
+  uint64_t s_full[2];           // MMA commit after QK: partial scores in buffer g
+  uint64_t s_empty[2];          // group g (4 arrivals) after reading its partial scores
+  uint64_t p_full[2];           // group g (4 arrivals) after writing P
   uint64_t p_free[2];           // MMA commit after PV of the tile: P buffer free, O stable
-  uint64_t x_full[kXBufs];      // 1 local arrival + kXBytes from the peer's st.async
+  uint64_t x_full[2];           // 1 local arrival + kXBytes of the peer group's st.async
+  uint64_t x_free[2];           // 4 arrivals of the peer's group g once it has read our push
+  uint64_t m_ready[2][4];       // group g, lane quarter q (1 arrival): running maximum published
   uint32_t vmask[kStages][2];   // valid positions of the tile in each stage (bit n of word n/32)
   uint32_t tmem_addr;
   int abort_flag;
 };
-static_assert(sizeof(AttendBars) <= 256, "barrier block");
+static_assert(sizeof(AttendBars) <= kBarBytes, "barrier block");
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Two floats to a pair of fp16 (round to nearest, saturated to +-65504 so a
+// huge score cannot turn into inf - inf = NaN); `lo` goes to the low half.
+__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t u) {
+  __half2 h;
+  memcpy(&h, &u, 4);
+  return __half22float2(h);
 }
 
 // Optional pipeline trace (compile with -DMLA_TRACE): per-tile clock64()
@@ -242,13 +257,16 @@ enum TraceEvent {
   kTrQkIssued,         // MMA thread: QK of the tile issued and committed
   kTrPvStart,          // MMA thread: PV of the tile starts issuing
   kTrPvIssued,         // MMA thread: PV of the tile issued and committed
-  kTrXStart,           // exchange warp 8: partial scores of the tile available
-  kTrXPushed,          // exchange warp 8: partial scores pushed to the peer
-  kTrXArrived,         // exchange warp 8: peer's partial scores observed
-  kTrXSummed,          // exchange warp 8: scaled full scores written back
-  kTrSmStart,          // softmax warp 0: scores of the tile available
-  kTrSmRead,           // softmax warp 0: scores read, buffer released
-  kTrPWritten,         // softmax warp 0: P of the tile written, p_full arrived
+  kTrSmStart,          // softmax (lane 0 of the group's first warp): partial scores available
+  kTrSmPushed,         //   own half pushed to the peer
+  kTrSmArrived,        //   peer's half observed
+  kTrSmMax,            //   running maximum of the tile published
+  kTrPWritten,         //   P written, p_full arrived
+  kTrSmConverted,      //   own half read, reduced and rounded
+  kTrSmFreeOk,         //   peer buffer free
+  kTrSmSummed,         //   full scores and tile maximum formed
+  kTrSmReleased,       //   peer told that its push has been read
+  kTrSmMaxIn,          //   other group's running maximum received
   kTrEvents
 };
 constexpr int kTraceTiles = 512;
@@ -290,8 +308,8 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
   const uint32_t sX = smem_u32(smem + kOffX);
   const uint32_t sQs = smem_u32(smem + kOffQs);
   const uint32_t sQpe = smem_u32(smem + kOffQpe);
-  float* tmax = reinterpret_cast<float*>(smem + kOffTmax);  // [tile parity][head]
-  float* red = reinterpret_cast<float*>(smem + kOffRed);    // [half][head]
+  float* mslot = reinterpret_cast<float*>(smem + kOffMslot);  // [group][head]
+  float* red = reinterpret_cast<float*>(smem + kOffRed);      // [l | m][group][head]
   AttendBars* bars = reinterpret_cast<AttendBars*>(smem + kOffBar);
   const AbortState ab{&bars->abort_flag, d_status};
   const float c2 = scale * 1.4426950408889634f;  // scores to log2 units
@@ -305,14 +323,13 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars->s_full[i]), 1);
-      mbar_init(smem_u32(&bars->s_sum[i]), kXchgWarps);
-      mbar_init(smem_u32(&bars->s_empty[i]), kSoftmaxWarps);
-      mbar_init(smem_u32(&bars->p_full[i]), kSoftmaxWarps);
+      mbar_init(smem_u32(&bars->s_empty[i]), 4);
+      mbar_init(smem_u32(&bars->p_full[i]), 4);
       mbar_init(smem_u32(&bars->p_free[i]), 1);
-    }
-    for (int i = 0; i < kXBufs; ++i) {
       mbar_init(smem_u32(&bars->x_full[i]), 1);
-      mbar_arrive_expect_tx(smem_u32(&bars->x_full[i]), kXBytes);  // armed for tiles 0..kXBufs-1
+      mbar_arrive_expect_tx(smem_u32(&bars->x_full[i]), kXBytes);  // armed for the group's first tile
+      mbar_init(smem_u32(&bars->x_free[i]), 4);
+      for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&bars->m_ready[i][q]), 1);
     }
     fence_mbarrier_init_cluster();
   }
@@ -327,7 +344,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
 
   if (warp >= kGatherWarp0) {
     // ------------------------------------------------------------ gather
-    // Gather warp g owns stage g and tiles g, g+3, g+6, ...; lane l handles
+    // Gather warp g owns stage g and tiles g, g+4, g+8, ...; lane l handles
     // positions l and l+32 of a tile.  Latent: one position per instruction
     // (32 lanes x 16 bytes = this CTA's 256 columns); rotary: eight positions
     // per instruction (this CTA's 32 columns).  A tile is published
@@ -376,8 +393,6 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
         MLA_TRACE_STAMP(kTrGatherLanded, j);
       }
     };
-    // this warp's next two tiles, statically indexed (a register copy of a
-    // pending load would wait for the load)
     // Rows of this warp's next tile are pulled into L2 while the tile ahead
     // of it is still in use, so its copies hit L2 once the stage frees.
     auto prefetch_tile = [&](int idx0, int idx1) {
@@ -392,6 +407,8 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
         }
       }
     };
+    // this warp's next two tiles, statically indexed (a register copy of a
+    // pending load would wait for the load)
     int a0 = load_idx(g, 0), a1 = load_idx(g, 1);
     int b0 = load_idx(g + kStages, 0), b1 = load_idx(g + kStages, 1);
     for (int j = g; j < n_tiles; j += 2 * kStages) {
@@ -484,82 +501,21 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       }
     }
     __syncwarp();
-  } else if (warp >= kXchgWarp0) {
-    // ------------------------------------------------------------ exchange
-    const int qd = warp & 3;
-    const int i = qd * 32 + lane;  // head
-    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
-    const bool leader = (warp == kXchgWarp0 && lane == 0);
-    uint32_t x_peer[kXBufs], xfull_peer[kXBufs];
-#pragma unroll
-    for (int u = 0; u < kXBufs; ++u) {
-      x_peer[u] = cluster_map(sX + u * kXBytes, peer);
-      xfull_peer[u] = cluster_map(smem_u32(&bars->x_full[u]), peer);
-    }
-    for (int j = 0; j < n_tiles; ++j) {
-      const int u = j % kXBufs;
-      const uint32_t sbuf = tmem + lane_base + kColS + (j & 1) * kNt;
-      wait(smem_u32(&bars->s_full[j & 1]), (j >> 1) & 1, ab);
-      tc_fence_after();
-      if (leader) MLA_TRACE_STAMP(kTrXStart, j);
-      uint32_t sv[64];
-      tmem_ld32(sbuf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(sbuf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tmem_wait_ld();
-#pragma unroll
-      for (int q = 0; q < 16; ++q)
-        st_async_v4(x_peer[u] + (uint32_t)((q * kH + i) * 16), sv[4 * q], sv[4 * q + 1], sv[4 * q + 2],
-                    sv[4 * q + 3], xfull_peer[u]);
-      if (leader) MLA_TRACE_STAMP(kTrXPushed, j);
-      // valid positions of tile j (the stage cannot be refilled before PV(j))
-      const int st = j % kStages;
-      wait(smem_u32(&bars->kv_full[st]), (j / kStages) & 1, ab);
-      const uint32_t vm0 = *reinterpret_cast<volatile uint32_t*>(&bars->vmask[st][0]);
-      const uint32_t vm1 = *reinterpret_cast<volatile uint32_t*>(&bars->vmask[st][1]);
-      wait(smem_u32(&bars->x_full[u]), (j / kXBufs) & 1, ab);
-      if (leader) {
-        MLA_TRACE_STAMP(kTrXArrived, j);
-        mbar_arrive_expect_tx(smem_u32(&bars->x_full[u]), kXBytes);  // re-arm for tile j + kXBufs
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const float4 o = *reinterpret_cast<const float4*>(smem + kOffX + u * kXBytes + (q * kH + i) * 16);
-        const float po[4] = {o.x, o.y, o.z, o.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int t = 4 * q + e;
-          const bool v = (((t < 32) ? vm0 : vm1) >> (t & 31)) & 1u;
-          const float x = v ? (__uint_as_float(sv[t]) + po[e]) * c2 : -INFINITY;  // log2 units; masked -> -inf
-          mx = fmaxf(mx, x);
-          sv[t] = __float_as_uint(x);
-        }
-      }
-      tmax[(j & 1) * kH + i] = mx;
-      tmem_st32(sbuf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_st32(sbuf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->s_sum[j & 1]));
-      if (leader) MLA_TRACE_STAMP(kTrXSummed, j);
-    }
   } else {
     // ------------------------------------------------------------ softmax
+    const int grp = warp >> 2;      // tiles grp, grp+2, ...
     const int qd = warp & 3;        // TMEM lane quarter
-    const int hf = warp >> 2;       // positions [32hf, 32hf+32) of every tile
     const int i = qd * 32 + lane;   // head
-    const bool leader = (warp == 0 && lane == 0);
+    const bool leader = (qd == 0 && lane == 0);
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
-    float m_used = -INFINITY, l_part = 0.f;
 
-    // This CTA's half of the query: latent columns 0..127 into TMEM (warp
-    // half 0), latent columns 128..255 into shared memory as two 128B-
-    // swizzled K-major blocks and the 32 rotary values as a 64B-swizzled
-    // K-major row (warp half 1).
+    // This CTA's half of the query: latent columns 0..127 into TMEM (group
+    // 0), latent columns 128..255 into shared memory as two 128B-swizzled
+    // K-major blocks and the 32 rotary values as a 64B-swizzled K-major row
+    // (group 1).
     {
       const uint4* ql = reinterpret_cast<const uint4*>(q_lat + ((size_t)b * kH + i) * kDl + rank * 256);
-      if (hf == 0) {
+      if (grp == 0) {
 #pragma unroll
         for (int part = 0; part < 2; ++part) {  // 64 latent values = 32 columns each
           uint32_t r[32];
@@ -598,80 +554,196 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));
     }
 
-    for (int j = 0; j < n_tiles; ++j) {
-      // scaled, masked scores of tile j (this warp's 32 positions) and the
-      // row maxima over all 64, from the exchange warps
-      uint32_t sv[32];
-      wait(smem_u32(&bars->s_sum[j & 1]), (j >> 1) & 1, ab);
+    const uint32_t sbuf = tmem + lane_base + kColS + grp * kNt;
+    const uint32_t pbuf = tmem + lane_base + kColP + grp * (kNt / 2);
+    const uint32_t x_mine = sX + grp * kXBytes;              // the peer's half arrives here
+    const uint32_t x_peer = cluster_map(x_mine, peer);       // our half goes there
+    const uint32_t xfull_peer = cluster_map(smem_u32(&bars->x_full[grp]), peer);
+    const uint32_t xfree_peer = cluster_map(smem_u32(&bars->x_free[grp]), peer);
+    float m_cur = -INFINITY;  // running maximum as of this group's last tile (log2 units)
+    float l_part = 0.f;       // this group's share of the row sum, relative to m_cur
+
+    int it = 0;  // this group's tile counter: tile j = 2 it + grp
+    for (int j = grp; j < n_tiles; j += 2, ++it) {
+      // partial scores of tile j: read, release the buffer
+      wait(smem_u32(&bars->s_full[grp]), it & 1, ab);
       tc_fence_after();
       if (leader) MLA_TRACE_STAMP(kTrSmStart, j);
-      tmem_ld32(tmem + lane_base + kColS + (j & 1) * kNt + 32 * hf, sv);
-      const float mx = tmax[(j & 1) * kH + i];
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[j & 1]));
-      if (leader) MLA_TRACE_STAMP(kTrSmRead, j);
+      // valid positions of tile j (the stage cannot be refilled before PV(j))
+      const int st = j % kStages;
+      wait(smem_u32(&bars->kv_full[st]), (j / kStages) & 1, ab);
+      const uint32_t vm0 = *reinterpret_cast<volatile uint32_t*>(&bars->vmask[st][0]);
+      const uint32_t vm1 = *reinterpret_cast<volatile uint32_t*>(&bars->vmask[st][1]);
+      // Our half in log2 units, as fp16 relative to its own maximum over the
+      // tile (sent exactly, in fp32, beside it): the rounding then scales with
+      // the spread of the scores inside the tile, not with their size.
+      // Padding positions become -inf, which the peer's sum carries along.
+      uint32_t hv[32];
+      float off;
+      {
+        uint32_t sv[64];
+        tmem_ld32(sbuf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(sbuf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[grp]));
+        float om = __uint_as_float(sv[0]);
+#pragma unroll
+        for (int t = 1; t < 64; ++t) om = fmaxf(om, __uint_as_float(sv[t]));
+        off = om * c2;  // c2 > 0: the maximum of the scaled values
+#pragma unroll
+        for (int t = 0; t < 32; ++t)
+          hv[t] = pack_f16x2_sat(fmaf(__uint_as_float(sv[2 * t]), c2, -off),
+                                 fmaf(__uint_as_float(sv[2 * t + 1]), c2, -off));
+      }
+      if ((vm0 & vm1) != 0xffffffffu) {  // a tile with padding (the tail of a split)
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          const uint32_t w = (t < 16) ? vm0 : vm1;
+          const uint32_t keep = (((w >> ((2 * t) & 31)) & 1u) ? 0x0000ffffu : 0u) |
+                                (((w >> ((2 * t + 1) & 31)) & 1u) ? 0xffff0000u : 0u);
+          hv[t] = (hv[t] & keep) | (0xfc00fc00u & ~keep);  // fp16 -inf where masked
+        }
+      }
+      // push our half into the peer's buffer (free once the peer has read our
+      // previous push from it)
+      if (leader) MLA_TRACE_STAMP(kTrSmConverted, j);
+      if (it > 0) wait_cluster(smem_u32(&bars->x_free[grp]), (it - 1) & 1, ab);
+      if (leader) MLA_TRACE_STAMP(kTrSmFreeOk, j);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        st_async_v4(x_peer + (uint32_t)((q * kH + i) * 16), hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3],
+                    xfull_peer);
+      st_async_b32(x_peer + (uint32_t)(kXHalves + i * 4), __float_as_uint(off), xfull_peer);
+      if (leader) MLA_TRACE_STAMP(kTrSmPushed, j);
 
-      // The running maximum of a row moves only when the tile's maximum
-      // exceeds it by more than 2^8 (so p <= 256 otherwise).  The TMEM
-      // accesses are warp-collective, so the whole warp rescales when any of
-      // its rows must (both warps of a pair decide alike); rows that keep
-      // their maximum use alpha = 1.  Each warp of the pair rescales half of
-      // the row.
-      const bool grow = mx > m_used + kRescaleThreshold;
-      const float alpha = grow ? ((m_used == -INFINITY) ? 0.f : ex2_approx(m_used - mx)) : 1.f;
+      // The peer's half.  Scores relative to base = off + off_peer, summed
+      // as fp16 pairs: both CTAs add the same two values (addition commutes),
+      // so their scores and everything after them are bitwise identical.
+      wait(smem_u32(&bars->x_full[grp]), it & 1, ab);
+      if (qd == 0 && lane == 0) {
+        MLA_TRACE_STAMP(kTrSmArrived, j);
+        mbar_arrive_expect_tx(smem_u32(&bars->x_full[grp]), kXBytes);  // re-arm for tile j + 2
+      }
+      float off_peer;
+      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(off_peer) : "r"(x_mine + (uint32_t)(kXHalves + i * 4)) : "memory");
+      const float base = off + off_peer;
+      uint32_t sh[32];
+      __half2 hmx = __halves2half2(__ushort_as_half(0xfc00u), __ushort_as_half(0xfc00u));
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint32_t o[4];
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+                     : "r"(x_mine + (uint32_t)((q * kH + i) * 16))
+                     : "memory");
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          __half2 a, p2;
+          memcpy(&a, &hv[4 * q + e], 4);
+          memcpy(&p2, &o[e], 4);
+          const __half2 sum = __hadd2(a, p2);
+          hmx = __hmax2(hmx, sum);
+          memcpy(&sh[4 * q + e], &sum, 4);
+        }
+      }
+      const float2 hm = __half22float2(hmx);
+      const float mx = fmaxf(hm.x, hm.y) + base;  // the tile maximum (-inf if all masked)
+      if (leader) MLA_TRACE_STAMP(kTrSmSummed, j);
+      // Every lane has consumed its loads of the peer's push (the sums above
+      // use them), so the peer may overwrite the buffer with tile j + 2.  A
+      // relaxed arrival: a release here would wait for our own pushes in
+      // flight to the peer.
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote_relaxed(xfree_peer);
+      if (leader) MLA_TRACE_STAMP(kTrSmReleased, j);
+
+      // Running maximum.  It moves only when a tile's maximum exceeds it by
+      // more than 2^8 (so p <= 256 otherwise).  The other group hands over
+      // its value after tile j-1; this group's row sum is brought to it.
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        wait(smem_u32(&bars->m_ready[grp ^ 1][qd]), ((j - 1) >> 1) & 1, ab);
+        m_prev = mslot[(grp ^ 1) * kH + i];
+      }
+      if (leader) MLA_TRACE_STAMP(kTrSmMaxIn, j);
+      if (m_prev != m_cur) {
+        l_part = (m_cur == -INFINITY) ? 0.f : l_part * ex2_approx(m_cur - m_prev);
+        m_cur = m_prev;
+      }
+      const bool grow = mx > m_cur + kRescaleThreshold;
+      const float alpha = grow ? ((m_cur == -INFINITY) ? 0.f : ex2_approx(m_cur - mx)) : 1.f;
+      if (grow) m_cur = mx;
+      mslot[grp * kH + i] = m_cur;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->m_ready[grp][qd]));
+      if (leader) MLA_TRACE_STAMP(kTrSmMax, j);
+
+      // The TMEM accesses are warp-collective, so the whole warp rescales
+      // when any of its rows must; rows that keep their maximum use alpha = 1.
       if (__any_sync(0xffffffffu, grow) && j > 0) {
         // PV(j-1) (and so every earlier MMA) must have finished before O is
-        // rescaled in place
+        // rescaled in place; PV(j) waits for this group's P.
         wait(smem_u32(&bars->p_free[(j - 1) & 1]), ((j - 1) >> 1) & 1, ab);
         tc_fence_after();
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          const uint32_t col = kColO + 128 * hf + cc * 32;
-          uint32_t ov[32];
-          tmem_ld32(tmem + lane_base + col, ov);
+        for (int cc = 0; cc < 16; ++cc) {
+          const uint32_t col = kColO + cc * 16;
+          uint32_t ov[16];
+          tmem_ld16(tmem + lane_base + col, ov);
           tmem_wait_ld();
 #pragma unroll
-          for (int t = 0; t < 32; ++t) ov[t] = __float_as_uint(__uint_as_float(ov[t]) * alpha);
-          tmem_st32(tmem + lane_base + col, ov);
+          for (int t = 0; t < 16; ++t) ov[t] = __float_as_uint(__uint_as_float(ov[t]) * alpha);
+          tmem_st16(tmem + lane_base + col, ov);
         }
         tmem_wait_st();
       }
       l_part *= alpha;
-      if (grow) m_used = mx;
 
       // Masked positions hold -inf and give exp2(-inf) = 0.  While a row has
       // seen no valid position its maximum is still -inf; subtracting 0 then
       // keeps every masked term at exactly 0 instead of exp2(NaN).
-      const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
-      uint32_t pk[16];
+      const float m_sub = (m_cur == -INFINITY) ? 0.f : m_cur;
+      const float csub = m_sub - base;  // s - m_sub = s_rel - csub
+      // this group's P buffer was last read by PV(j-2)
+      if (it > 0) wait(smem_u32(&bars->p_free[grp]), (it - 1) & 1, ab);
+      tc_fence_after();
       float lt = 0.f;
 #pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        const float p0 = ex2_approx(__uint_as_float(sv[2 * t]) - m_sub);
-        const float p1 = ex2_approx(__uint_as_float(sv[2 * t + 1]) - m_sub);
-        pk[t] = pack_bf16x2(p0, p1);
-        lt += p0 + p1;
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const float2 f = unpack_f16x2(sh[16 * hh + t]);
+          const float p0 = ex2_approx(f.x - csub);
+          const float p1 = ex2_approx(f.y - csub);
+          pk[t] = pack_bf16x2(p0, p1);
+          lt += p0 + p1;
+        }
+        tmem_st16(pbuf + 16 * hh, pk);
       }
       l_part += lt;
-      // P buffer j&1 was last read by PV(j-2)
-      if (j >= 2) wait(smem_u32(&bars->p_free[j & 1]), ((j >> 1) - 1) & 1, ab);
-      tc_fence_after();
-      tmem_st16(tmem + lane_base + kColP + (j & 1) * (kNt / 2) + 16 * hf, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[j & 1]));
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[grp]));
       if (leader) MLA_TRACE_STAMP(kTrPWritten, j);
     }
 
-    // epilogue: row sums of the pair combined, normalised O half and the
-    // split's log-sum-exp
-    red[hf * kH + i] = l_part;
-    named_bar_sync(1 + qd, 64);
-    const float l_sum = l_part + red[(hf ^ 1) * kH + i];
-    float* orow = o_part + (((size_t)b * n_split + split) * kH + i) * kDl + rank * 256 + 128 * hf;
+    // epilogue: both groups' row sums brought to the final maximum (the
+    // larger of the two: the maximum never decreases), normalised O half and
+    // the split's log-sum-exp
+    red[grp * kH + i] = l_part;
+    red[(2 + grp) * kH + i] = m_cur;
+    named_bar_sync(1 + qd, 64);  // warps qd and qd + 4
+    const float l_o = red[(grp ^ 1) * kH + i];
+    const float m_o = red[(2 + (grp ^ 1)) * kH + i];
+    const float m_fin = fmaxf(m_cur, m_o);
+    const float l_a = (m_cur == -INFINITY) ? 0.f : l_part * ex2_approx(m_cur - m_fin);
+    const float l_b = (m_o == -INFINITY) ? 0.f : l_o * ex2_approx(m_o - m_fin);
+    const float l_sum = l_a + l_b;  // the same sum in both groups (fp32 addition commutes)
+    float* orow = o_part + (((size_t)b * n_split + split) * kH + i) * kDl + rank * 256 + 128 * grp;
     if (n_tiles > 0) {
       // the last PV done implies every MMA of the split is done
       wait(smem_u32(&bars->p_free[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, ab);
@@ -682,7 +754,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     for (int cc = 0; cc < 4; ++cc) {
       uint32_t ov[32];
       if (n_tiles > 0) {
-        tmem_ld32(tmem + lane_base + kColO + 128 * hf + cc * 32, ov);
+        tmem_ld32(tmem + lane_base + kColO + 128 * grp + cc * 32, ov);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -695,9 +767,9 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
         *reinterpret_cast<float4*>(orow + cc * 32 + t) = v;
       }
     }
-    if (rank == 0 && hf == 0) {
+    if (rank == 0 && grp == 0) {
       lse_part[((size_t)b * n_split + split) * kH + i] =
-          l_sum > 0.f ? (m_used + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
+          l_sum > 0.f ? (m_fin + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
     }
   }
 
@@ -709,7 +781,6 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
   cluster_sync();
 }
-
 // =============================================================================
 // combine_value_up_kernel
 //
