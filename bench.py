@@ -233,7 +233,10 @@ def gpu_arm(args, rank, world, device):
 
     # ---- per-kernel live timing (same stream, back-to-back launches, sets rotate)
     q_lat = [torch.empty((B, 128, 512), dtype=torch.bfloat16, device=device) for _ in sets]
-    o_part = torch.empty((B, n_split, 128, 512), dtype=torch.float32, device=device)
+    # the attention kernel's per-split output: f32 partials, or the bf16 mixed
+    # latent when each row is a single split
+    o_part = (torch.empty((B, 128, 512), dtype=torch.bfloat16, device=device) if n_split == 1 else
+              torch.empty((B, n_split, 128, 512), dtype=torch.float32, device=device))
     lse_part = torch.empty((B, n_split, 128), dtype=torch.float32, device=device)
     sv = ctypes.c_void_p(stream.cuda_stream)
 

@@ -73,8 +73,9 @@ const char* mla_status_string(int status);
 int mla_num_splits(int B, int K);
 
 /* Bytes of scratch `mla_sparse_decode` needs for these sizes on the current
- * device: the absorbed queries (bf16 [B,128,512]) and the per-split partial
- * outputs (f32 [B,splits,128,512] plus f32 [B,splits,128]).  Returns 0 for
+ * device: the absorbed queries (bf16 [B,128,512]), the per-split outputs of
+ * mla_sparse_attend (see there: f32 [B,splits,128,512], or bf16 [B,128,512]
+ * with one split) and their log-sum-exps (f32 [B,splits,128]).  Returns 0 for
  * invalid sizes. */
 size_t mla_sparse_decode_workspace_size(int B, int K, int S_max);
 
@@ -114,25 +115,30 @@ int mla_absorb_q(const void* q_nope, const void* wkv_b, void* q_lat, int B, cuda
  * Steps "scores" .. "mix" for every (row, split) (model.py 596-605), the
  * key positions of row b being split into `n_split` contiguous ranges of index
  * slots:
- *   o_part[b,s,h,:]  f32 [B,n_split,128,512]  softmax-normalised mix of the
- *                    cached latents over the valid positions of split s
+ *   o_part           n_split > 1: f32 [B,n_split,128,512], o_part[b,s,h,:] =
+ *                    softmax-normalised mix of the cached latents over the
+ *                    valid positions of split s;
+ *                    n_split == 1: bf16 [B,128,512], the mixed latent
+ *                    O~[b,h,:] itself (rounded to bf16, the value-up operand)
  *   lse_part[b,s,h]  f32 [B,n_split,128]      log-sum-exp of the split's
  *                    scaled scores (-inf when the split has no valid index)
  *   q_lat bf16 [B,128,512] (from mla_absorb_q), the other inputs as above.
  * n_split must equal mla_num_splits(B, K).
  */
 int mla_sparse_attend(const void* q_lat, const void* q_pe, const void* kv_cache, const void* pe_cache,
-                      const int32_t* end_pos, const int32_t* topk_idx, float scale, float* o_part,
+                      const int32_t* end_pos, const int32_t* topk_idx, float scale, void* o_part,
                       float* lse_part, int B, int K, int S_max, int n_split, int* d_status, cudaStream_t stream);
 
 /*
- * Steps "combine" and "value-up" (model.py 605-606):
+ * Steps "combine" and "value-up" (model.py 605-606), o_part and lse_part in
+ * the layout mla_sparse_attend writes for this n_split:
  *   O~[b,h,:] = sum_s exp(lse_part[b,s,h] - L) o_part[b,s,h,:],
- *   L = log sum_s exp(lse_part[b,s,h]),
+ *   L = log sum_s exp(lse_part[b,s,h])          (n_split > 1; with one split
+ *                                                O~ = o_part, L = lse_part),
  *   out[b,h,e] = bf16( sum_c bf16(O~[b,h,c]) * wkv_b[h*256 + 128 + e, c] ),
  *   lse_out[b,h] = L (optional).
  */
-int mla_combine_value_up(const float* o_part, const float* lse_part, const void* wkv_b, void* out,
+int mla_combine_value_up(const void* o_part, const float* lse_part, const void* wkv_b, void* out,
                          float* lse_out, int B, int n_split, cudaStream_t stream);
 
 /*

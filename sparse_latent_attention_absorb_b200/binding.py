@@ -144,9 +144,19 @@ def mla_absorb_q(q_nope, wkv_b, q_lat=None, stream=None):
     return q_lat
 
 
+def _o_part_spec(B: int, n_split: int):
+    """Shape and dtype of mla_sparse_attend's o_part for this split count."""
+    if n_split == 1:
+        return (B, H, D_LAT), torch.bfloat16
+    return (B, n_split, H, D_LAT), torch.float32
+
+
 def mla_sparse_attend(q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, scale, o_part=None, lse_part=None,
                       d_status=None, stream=None):
-    """Per-split partial outputs; returns (o_part [B,S,128,512] f32, lse_part [B,S,128] f32)."""
+    """Per-split outputs; returns (o_part, lse_part [B,S,128] f32).
+
+    o_part is f32 [B,S,128,512] (normalised mix per split) when S > 1, and the
+    bf16 mixed latent [B,128,512] when each row is one split (S == 1)."""
     lib = load_library()
     B, S_max, K = q_lat.shape[0], kv_cache.shape[1], topk_idx.shape[1]
     n_split = num_splits(B, K)
@@ -158,11 +168,12 @@ def mla_sparse_attend(q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, scale,
     _check(end_pos, "end_pos", torch.int32, (B,))
     _check(topk_idx, "topk_idx", torch.int32, (B, K))
     dev = q_lat.device
+    o_shape, o_dtype = _o_part_spec(B, n_split)
     if o_part is None:
-        o_part = torch.empty((B, n_split, H, D_LAT), dtype=torch.float32, device=dev)
+        o_part = torch.empty(o_shape, dtype=o_dtype, device=dev)
     if lse_part is None:
         lse_part = torch.empty((B, n_split, H), dtype=torch.float32, device=dev)
-    _check(o_part, "o_part", torch.float32, (B, n_split, H, D_LAT))
+    _check(o_part, "o_part", o_dtype, o_shape)
     _check(lse_part, "lse_part", torch.float32, (B, n_split, H))
     rc = lib.mla_sparse_attend(_ptr(q_lat), _ptr(q_pe), _ptr(kv_cache), _ptr(pe_cache), _ptr(end_pos),
                                _ptr(topk_idx), float(scale), _ptr(o_part), _ptr(lse_part), B, K, S_max, n_split,
@@ -172,10 +183,12 @@ def mla_sparse_attend(q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, scale,
 
 
 def mla_combine_value_up(o_part, lse_part, wkv_b, out=None, lse_out=None, stream=None):
+    """Merge of the splits and W_UV; o_part / lse_part as mla_sparse_attend returns them."""
     lib = load_library()
-    B, n_split = o_part.shape[0], o_part.shape[1]
+    B, n_split = lse_part.shape[0], lse_part.shape[1]
     bf = torch.bfloat16
-    _check(o_part, "o_part", torch.float32, (B, n_split, H, D_LAT))
+    o_shape, o_dtype = _o_part_spec(B, n_split)
+    _check(o_part, "o_part", o_dtype, o_shape)
     _check(lse_part, "lse_part", torch.float32, (B, n_split, H))
     _check(wkv_b, "wkv_b", bf, (H * (D_NOPE + D_V), D_LAT))
     if out is None:

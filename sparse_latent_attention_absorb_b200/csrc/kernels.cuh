@@ -47,8 +47,10 @@ __device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* p) {
 // =============================================================================
 constexpr int kAbsorbNMax = 128;
 constexpr int kAbsorbSmemA = 2 * 64 * 128 * 2;                      // 32 KB
-constexpr int kAbsorbSmemB = 2 * kAbsorbNMax * 128;                  // 32 KB max
-constexpr int kAbsorbSmemBytes = kAbsorbSmemA + kAbsorbSmemB + 256 + kSmemAlignPad;  // + barriers
+// shared memory for a batch tile of n rows: W_UK chunk, q_nope tile, barriers
+// (sized to the tile so that four CTAs fit on an SM when n <= 64)
+__host__ __device__ constexpr int absorb_smem_bytes(int n) { return kAbsorbSmemA + 2 * n * 128 + 256 + kSmemAlignPad; }
+constexpr int kAbsorbSmemBytes = absorb_smem_bytes(kAbsorbNMax);
 
 __global__ void __launch_bounds__(128, 1)
 absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
@@ -62,7 +64,7 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + kAbsorbSmemA;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAbsorbSmemA + kAbsorbSmemB);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAbsorbSmemA + 2 * n_tile * 128);
   const uint32_t bar_load = smem_u32(&bars[0]);
   const uint32_t bar_mma = smem_u32(&bars[1]);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2]);
@@ -94,6 +96,7 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
     tma_load_2d(sA + 64 * 128 * 2, &tm_w, bar_load, chunk * 128 + 64, wrow);
     tma_load_3d(sB, &tm_q, bar_load, 0, h, b0);
     tma_load_3d(sB + n_tile * 128, &tm_q, bar_load, 64, h, b0);
+    grid_dep_launch();  // the attention kernel may start gathering
 
     wait(bar_load, 0, ab);
     tc_fence_after();
@@ -159,7 +162,8 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 //     group's TMEM buffer;
 //   * PV: O_r[h, its 256] += P[h,t] . kv[t, its 256]  (A = P from TMEM,
 //     B = the same gathered rows read M/N-major).
-// The split's normalised O and its log-sum-exp go to o_part / lse_part.
+// The split's normalised O and its log-sum-exp go to o_part / lse_part (O in
+// f32 per split; with a single split per row, the final O~ in bf16).
 //
 // Warp roles (416 threads): warps 0-3 softmax group 0 (even tiles), warps
 // 4-7 softmax group 1 (odd tiles), warp w covering TMEM lanes 32(w%4)..;
@@ -287,7 +291,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttendThreads, 1)
 sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat16* __restrict__ q_pe,
                      const __nv_bfloat16* __restrict__ kv_cache, const __nv_bfloat16* __restrict__ pe_cache,
                      const int32_t* __restrict__ end_pos, const int32_t* __restrict__ topk_idx, float scale,
-                     float* __restrict__ o_part, float* __restrict__ lse_part, int K, int S_max, int n_split,
+                     void* __restrict__ o_part, float* __restrict__ lse_part, int K, int S_max, int n_split,
                      int span, int* d_status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
@@ -341,6 +345,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
   cluster_sync();  // barriers of both CTAs initialised before any remote access
   tc_fence_after();
   const uint32_t tmem = bars->tmem_addr;
+  grid_dep_launch();  // the combine kernel may start loading its weights
 
   if (warp >= kGatherWarp0) {
     // ------------------------------------------------------------ gather
@@ -514,6 +519,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     // K-major blocks and the 32 rotary values as a 64B-swizzled K-major row
     // (group 1).
     {
+      grid_dep_wait();  // q_lat comes from the absorption kernel
       const uint4* ql = reinterpret_cast<const uint4*>(q_lat + ((size_t)b * kH + i) * kDl + rank * 256);
       if (grp == 0) {
 #pragma unroll
@@ -743,13 +749,15 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     const float l_a = (m_cur == -INFINITY) ? 0.f : l_part * ex2_approx(m_cur - m_fin);
     const float l_b = (m_o == -INFINITY) ? 0.f : l_o * ex2_approx(m_o - m_fin);
     const float l_sum = l_a + l_b;  // the same sum in both groups (fp32 addition commutes)
-    float* orow = o_part + (((size_t)b * n_split + split) * kH + i) * kDl + rank * 256 + 128 * grp;
     if (n_tiles > 0) {
       // the last PV done implies every MMA of the split is done
       wait(smem_u32(&bars->p_free[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, ab);
       tc_fence_after();
     }
     const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+    // A row of one split is final here: its mixed latent O~ goes out in bf16
+    // (the value-up operand); several splits keep f32 partials for the merge.
+    const size_t orow = (((size_t)b * n_split + split) * kH + i) * kDl + rank * 256 + 128 * grp;
 #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {
       uint32_t ov[32];
@@ -760,11 +768,24 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
 #pragma unroll
         for (int t = 0; t < 32; ++t) ov[t] = 0u;
       }
+      if (n_split == 1) {
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(o_part) + orow + cc * 32;
 #pragma unroll
-      for (int t = 0; t < 32; t += 4) {
-        float4 v = make_float4(__uint_as_float(ov[t]) * inv, __uint_as_float(ov[t + 1]) * inv,
-                               __uint_as_float(ov[t + 2]) * inv, __uint_as_float(ov[t + 3]) * inv);
-        *reinterpret_cast<float4*>(orow + cc * 32 + t) = v;
+        for (int t = 0; t < 32; t += 8) {
+          const uint4 v = make_uint4(pack_bf16x2(__uint_as_float(ov[t]) * inv, __uint_as_float(ov[t + 1]) * inv),
+                                     pack_bf16x2(__uint_as_float(ov[t + 2]) * inv, __uint_as_float(ov[t + 3]) * inv),
+                                     pack_bf16x2(__uint_as_float(ov[t + 4]) * inv, __uint_as_float(ov[t + 5]) * inv),
+                                     pack_bf16x2(__uint_as_float(ov[t + 6]) * inv, __uint_as_float(ov[t + 7]) * inv));
+          *reinterpret_cast<uint4*>(dst + t) = v;
+        }
+      } else {
+        float* dst = reinterpret_cast<float*>(o_part) + orow + cc * 32;
+#pragma unroll
+        for (int t = 0; t < 32; t += 4) {
+          const float4 v = make_float4(__uint_as_float(ov[t]) * inv, __uint_as_float(ov[t + 1]) * inv,
+                                       __uint_as_float(ov[t + 2]) * inv, __uint_as_float(ov[t + 3]) * inv);
+          *reinterpret_cast<float4*>(dst + t) = v;
+        }
       }
     }
     if (rank == 0 && grp == 0) {
@@ -785,11 +806,14 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
 // combine_value_up_kernel
 //
 // Per (head h, tile of up to 64 rows b):
-//   coefficients a_s = exp(lse_s - L) with L = log sum_s exp(lse_s);
-//   O~[b, :] = sum_s a_s o_part[b, s, h, :], rounded to bf16 into shared memory
-//   (K-major B operand, 128B-swizzled);
+//   with several splits: coefficients a_s = exp(lse_s - L) with
+//   L = log sum_s exp(lse_s); O~[b, :] = sum_s a_s o_part[b, s, h, :], rounded
+//   to bf16 into shared memory (K-major B operand, 128B-swizzled);
+//   with one split: O~ is already bf16 in memory and comes in by TMA;
 //   D[e, b] = sum_c W_UV[h, e, c] * O~[b, c]   (M = 128 value dims, K = 512)
 //   with W_UV[h] (128 KB) brought in by eight TMA boxes.
+// W_UV is requested before the wait on the attention kernel (programmatic
+// dependent launch), so the weight read overlaps the end of that kernel.
 // =============================================================================
 constexpr int kCombineNMax = 64;
 constexpr int kCombineMaxSplits = 128;
@@ -801,9 +825,10 @@ constexpr int kCombineThreads = 256;
 static_assert(kCombineSmemBytes <= 232448, "shared memory");
 
 __global__ void __launch_bounds__(kCombineThreads, 1)
-combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const float* __restrict__ o_part,
-                        const float* __restrict__ lse_part, __nv_bfloat16* __restrict__ out,
-                        float* __restrict__ lse_out, int B, int n_split, int n_tile, int* d_status) {
+combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_o,
+                        const void* __restrict__ o_part, const float* __restrict__ lse_part,
+                        __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out, int B, int n_split, int n_tile,
+                        int* d_status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -817,8 +842,9 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const float* _
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kCombineSmemA + kCombineSmemB + kCombineSmemCoef);
   const uint32_t bar_w = smem_u32(&bars[0]);
   const uint32_t bar_mma = smem_u32(&bars[1]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[3]);
+  const uint32_t bar_o = smem_u32(&bars[2]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[3]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[4]);
   const AbortState ab{abort_flag, d_status};
   const uint32_t tmem_cols = n_tile <= 32 ? 32u : 64u;
 
@@ -826,6 +852,7 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const float* _
     *abort_flag = 0;
     mbar_init(bar_w, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_o, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -843,50 +870,66 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const float* _
     const int wrow = h * kHeadRows + kDn;  // W_UV rows of head h
     for (int kb = 0; kb < 8; ++kb) tma_load_2d(sA + kb * 128 * 128, &tm_w, bar_w, kb * 64, wrow);
   }
+  grid_dep_wait();  // o_part / lse_part come from the attention kernel
 
-  // split weights, one row per thread
-  if (tid < rows) {
-    const int b = b0 + tid;
-    float mx = -INFINITY;
-    for (int s = 0; s < n_split; ++s) mx = fmaxf(mx, lse_part[((size_t)b * n_split + s) * kH + h]);
-    float total = 0.f;
-    for (int s = 0; s < n_split; ++s) {
-      const float l = lse_part[((size_t)b * n_split + s) * kH + h];
-      const float w = (mx == -INFINITY) ? 0.f : __expf(l - mx);
-      coef[tid * kCombineMaxSplits + s] = w;
-      total += w;
+  if (n_split == 1) {
+    // O~ rows b0.. of head h: eight boxes of 64 columns x n_tile rows (rows
+    // past B read as zero)
+    if (tid == 0) {
+      tma_prefetch_desc(&tm_o);
+      mbar_arrive_expect_tx(bar_o, 8 * n_tile * 128);
+      for (int kb = 0; kb < 8; ++kb) tma_load_3d(sB + kb * n_tile * 128, &tm_o, bar_o, kb * 64, h, b0);
     }
-    const float inv = total > 0.f ? 1.f / total : 0.f;
-    for (int s = 0; s < n_split; ++s) coef[tid * kCombineMaxSplits + s] *= inv;
-    if (lse_out) lse_out[(size_t)b * kH + h] = total > 0.f ? mx + __logf(total) : -INFINITY;
-  }
-  __syncthreads();
-
-  // merged O~ rows -> bf16 K-major operand (row n = batch row, 512 columns)
-  for (int it = tid; it < n_tile * 64; it += kCombineThreads) {
-    const int n = it >> 6, q = it & 63;  // q: 8-column chunk of the 512
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (n < rows) {
-      const int b = b0 + n;
+    if (tid < rows && lse_out) lse_out[(size_t)(b0 + tid) * kH + h] = lse_part[(size_t)(b0 + tid) * kH + h];
+  } else {
+    const float* o_f32 = static_cast<const float*>(o_part);
+    // split weights, one row per thread
+    if (tid < rows) {
+      const int b = b0 + tid;
+      float mx = -INFINITY;
+      for (int s = 0; s < n_split; ++s) mx = fmaxf(mx, lse_part[((size_t)b * n_split + s) * kH + h]);
+      float total = 0.f;
       for (int s = 0; s < n_split; ++s) {
-        const float a = coef[n * kCombineMaxSplits + s];
-        const float4* src = reinterpret_cast<const float4*>(o_part + (((size_t)b * n_split + s) * kH + h) * kDl + q * 8);
-        const float4 x0 = src[0], x1 = src[1];
-        acc[0] += a * x0.x; acc[1] += a * x0.y; acc[2] += a * x0.z; acc[3] += a * x0.w;
-        acc[4] += a * x1.x; acc[5] += a * x1.y; acc[6] += a * x1.z; acc[7] += a * x1.w;
+        const float l = lse_part[((size_t)b * n_split + s) * kH + h];
+        const float w = (mx == -INFINITY) ? 0.f : __expf(l - mx);
+        coef[tid * kCombineMaxSplits + s] = w;
+        total += w;
       }
+      const float inv = total > 0.f ? 1.f / total : 0.f;
+      for (int s = 0; s < n_split; ++s) coef[tid * kCombineMaxSplits + s] *= inv;
+      if (lse_out) lse_out[(size_t)b * kH + h] = total > 0.f ? mx + __logf(total) : -INFINITY;
     }
-    const uint32_t dst = sB + (q >> 3) * (n_tile * 128) + sw128_offset(n, q & 7);
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pack_bf16x2(acc[0], acc[1])),
-                 "r"(pack_bf16x2(acc[2], acc[3])), "r"(pack_bf16x2(acc[4], acc[5])),
-                 "r"(pack_bf16x2(acc[6], acc[7]))
-                 : "memory");
+    __syncthreads();
+
+    // merged O~ rows -> bf16 K-major operand (row n = batch row, 512 columns)
+    for (int it = tid; it < n_tile * 64; it += kCombineThreads) {
+      const int n = it >> 6, q = it & 63;  // q: 8-column chunk of the 512
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (n < rows) {
+        const int b = b0 + n;
+#pragma unroll 4
+        for (int s = 0; s < n_split; ++s) {
+          const float a = coef[n * kCombineMaxSplits + s];
+          const float4* src =
+              reinterpret_cast<const float4*>(o_f32 + (((size_t)b * n_split + s) * kH + h) * kDl + q * 8);
+          const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
+          acc[0] += a * x0.x; acc[1] += a * x0.y; acc[2] += a * x0.z; acc[3] += a * x0.w;
+          acc[4] += a * x1.x; acc[5] += a * x1.y; acc[6] += a * x1.z; acc[7] += a * x1.w;
+        }
+      }
+      const uint32_t dst = sB + (q >> 3) * (n_tile * 128) + sw128_offset(n, q & 7);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pack_bf16x2(acc[0], acc[1])),
+                   "r"(pack_bf16x2(acc[2], acc[3])), "r"(pack_bf16x2(acc[4], acc[5])),
+                   "r"(pack_bf16x2(acc[6], acc[7]))
+                   : "memory");
+    }
+    fence_proxy_async_smem();
   }
-  fence_proxy_async_smem();
   __syncthreads();
 
   if (tid == 0) {
     wait(bar_w, 0, ab);
+    if (n_split == 1) wait(bar_o, 0, ab);
     tc_fence_after();
     const uint32_t idesc = idesc_bf16_f32(128, n_tile, false, false);
     for (int k = 0; k < kDl / 16; ++k) {

@@ -114,6 +114,20 @@ int encode_q_nope(CUtensorMap* m, const void* q_nope, int B, int n_tile) {
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// The mixed latent O~ (single-split rows) as a 3-D bf16 tensor
+// {c: 512, h: 128, b: B}, boxes of 64 c x 1 head x n_tile rows, 128-byte
+// swizzle (rows past B read as zero).
+int encode_o_lat(CUtensorMap* m, const void* o_lat, int B, int n_tile) {
+  cuuint64_t dims[3] = {(cuuint64_t)kDl, (cuuint64_t)kH, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)kDl * 2, (cuuint64_t)kH * kDl * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)n_tile};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(o_lat), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- planning
 
 constexpr int kMaxB = 1 << 20;
@@ -145,8 +159,8 @@ WorkspaceLayout workspace_layout(int B, int n_split) {
   size_t off = 0;
   w.q_lat = off;
   off = round_up(off + (size_t)B * kH * kDl * 2, 256);
-  w.o_part = off;
-  off = round_up(off + (size_t)B * n_split * kH * kDl * 4, 256);
+  w.o_part = off;  // f32 partials per split, or bf16 O~ when a row is one split
+  off = round_up(off + (size_t)B * n_split * kH * kDl * (n_split == 1 ? 2 : 4), 256);
   w.lse_part = off;
   off = round_up(off + (size_t)B * n_split * kH * 4, 256);
   w.total = off;
@@ -155,6 +169,30 @@ WorkspaceLayout workspace_layout(int B, int n_split) {
 
 int launch_check() { return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
+// Launch with or without a programmatic dependency on the previous kernel in
+// the stream.  With one, the kernel may start before that kernel has finished
+// and must call grid_dep_wait() before it reads anything the other writes; the
+// decode step uses it only between its own kernels.
+template <typename... KArgs, typename... Args>
+int launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
+              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  return launch_check();
+}
+
 int launch_absorb(const void* q_nope, const void* wkv_b, void* q_lat, int B, int* d_status, cudaStream_t stream) {
   const int n_tile = B >= kAbsorbNMax ? kAbsorbNMax : ceil_div(B, 16) * 16;
   CUtensorMap tm_w, tm_q;
@@ -162,32 +200,35 @@ int launch_absorb(const void* q_nope, const void* wkv_b, void* q_lat, int B, int
   if ((rc = encode_wkv_b(&tm_w, wkv_b)) != MLA_OK) return rc;
   if ((rc = encode_q_nope(&tm_q, q_nope, B, n_tile)) != MLA_OK) return rc;
   dim3 grid(kDl / 128, kH, ceil_div(B, kAbsorbNMax));
-  absorb_kernel<<<grid, 128, kAbsorbSmemBytes, stream>>>(tm_w, tm_q, static_cast<__nv_bfloat16*>(q_lat), B, n_tile, d_status);
-  return launch_check();
+  return launch_ex(absorb_kernel, grid, dim3(128), absorb_smem_bytes(n_tile), stream, false, tm_w, tm_q,
+                   static_cast<__nv_bfloat16*>(q_lat), B, n_tile, d_status);
 }
 
 int launch_attend(const void* q_lat, const void* q_pe, const void* kv_cache, const void* pe_cache,
-                  const int32_t* end_pos, const int32_t* topk_idx, float scale, float* o_part, float* lse_part, int B,
-                  int K, int S_max, int n_split, int span, int* d_status, cudaStream_t stream) {
+                  const int32_t* end_pos, const int32_t* topk_idx, float scale, void* o_part, float* lse_part, int B,
+                  int K, int S_max, int n_split, int span, int* d_status, cudaStream_t stream, bool pdl) {
   const long long ctas = 2LL * B * n_split;
   if (ctas > 0x7fffffffLL) return MLA_ERR_INVALID_ARG;
-  sparse_attend_kernel<<<(unsigned)ctas, kAttendThreads, kAttendSmemBytes, stream>>>(
-      static_cast<const __nv_bfloat16*>(q_lat), static_cast<const __nv_bfloat16*>(q_pe),
-      static_cast<const __nv_bfloat16*>(kv_cache), static_cast<const __nv_bfloat16*>(pe_cache), end_pos, topk_idx,
-      scale, o_part, lse_part, K, S_max, n_split, span, d_status);
-  return launch_check();
+  return launch_ex(sparse_attend_kernel, dim3((unsigned)ctas), dim3(kAttendThreads), kAttendSmemBytes, stream, pdl,
+                   static_cast<const __nv_bfloat16*>(q_lat), static_cast<const __nv_bfloat16*>(q_pe),
+                   static_cast<const __nv_bfloat16*>(kv_cache), static_cast<const __nv_bfloat16*>(pe_cache), end_pos,
+                   topk_idx, scale, o_part, lse_part, K, S_max, n_split, span, d_status);
 }
 
-int launch_combine(const float* o_part, const float* lse_part, const void* wkv_b, void* out, float* lse_out, int B,
-                   int n_split, int* d_status, cudaStream_t stream) {
+int launch_combine(const void* o_part, const float* lse_part, const void* wkv_b, void* out, float* lse_out, int B,
+                   int n_split, int* d_status, cudaStream_t stream, bool pdl) {
   const int n_tile = B >= kCombineNMax ? kCombineNMax : ceil_div(B, 16) * 16;
-  CUtensorMap tm_w;
+  CUtensorMap tm_w, tm_o;
   int rc;
   if ((rc = encode_wkv_b(&tm_w, wkv_b)) != MLA_OK) return rc;
+  if (n_split == 1) {
+    if ((rc = encode_o_lat(&tm_o, o_part, B, n_tile)) != MLA_OK) return rc;
+  } else {
+    tm_o = tm_w;  // unused
+  }
   dim3 grid(kH, ceil_div(B, kCombineNMax));
-  combine_value_up_kernel<<<grid, kCombineThreads, kCombineSmemBytes, stream>>>(
-      tm_w, o_part, lse_part, static_cast<__nv_bfloat16*>(out), lse_out, B, n_split, n_tile, d_status);
-  return launch_check();
+  return launch_ex(combine_value_up_kernel, grid, dim3(kCombineThreads), kCombineSmemBytes, stream, pdl, tm_w, tm_o,
+                   o_part, lse_part, static_cast<__nv_bfloat16*>(out), lse_out, B, n_split, n_tile, d_status);
 }
 
 int prepare(DeviceInfo** info) {
@@ -260,7 +301,7 @@ extern "C" int mla_absorb_q(const void* q_nope, const void* wkv_b, void* q_lat, 
 }
 
 extern "C" int mla_sparse_attend(const void* q_lat, const void* q_pe, const void* kv_cache, const void* pe_cache,
-                                 const int32_t* end_pos, const int32_t* topk_idx, float scale, float* o_part,
+                                 const int32_t* end_pos, const int32_t* topk_idx, float scale, void* o_part,
                                  float* lse_part, int B, int K, int S_max, int n_split, int* d_status,
                                  cudaStream_t stream) {
   const void* ptrs[] = {q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, o_part, lse_part};
@@ -274,10 +315,10 @@ extern "C" int mla_sparse_attend(const void* q_lat, const void* q_pe, const void
   plan_splits(B, K, info->sm_count, &want, &span);
   if (n_split != want) return MLA_ERR_INVALID_ARG;
   return launch_attend(q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, scale, o_part, lse_part, B, K, S_max,
-                       n_split, span, d_status, stream);
+                       n_split, span, d_status, stream, false);
 }
 
-extern "C" int mla_combine_value_up(const float* o_part, const float* lse_part, const void* wkv_b, void* out,
+extern "C" int mla_combine_value_up(const void* o_part, const float* lse_part, const void* wkv_b, void* out,
                                     float* lse_out, int B, int n_split, cudaStream_t stream) {
   if (!o_part || !lse_part || !wkv_b || !out) return MLA_ERR_INVALID_ARG;
   if (!aligned16(o_part) || !aligned16(lse_part) || !aligned16(wkv_b) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
@@ -286,7 +327,7 @@ extern "C" int mla_combine_value_up(const float* o_part, const float* lse_part, 
   DeviceInfo* info = nullptr;
   int rc = prepare(&info);
   if (rc != MLA_OK) return rc;
-  return launch_combine(o_part, lse_part, wkv_b, out, lse_out, B, n_split, nullptr, stream);
+  return launch_combine(o_part, lse_part, wkv_b, out, lse_out, B, n_split, nullptr, stream, false);
 }
 
 extern "C" int mla_sparse_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
@@ -309,14 +350,19 @@ extern "C" int mla_sparse_decode(const void* q_nope, const void* q_pe, const voi
     return MLA_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* q_lat = ws + wl.q_lat;
-  float* o_part = reinterpret_cast<float*>(ws + wl.o_part);
+  void* o_part = ws + wl.o_part;
   float* lse_part = reinterpret_cast<float*>(ws + wl.lse_part);
 
+  // The attention and combine kernels depend programmatically on the kernel
+  // before them: each starts while its predecessor drains and waits for it
+  // only where it reads that kernel's output.  The absorption kernel is an
+  // ordinary launch, so all earlier work in the stream (whatever wrote the
+  // caches and indices) has finished before any of the three starts.
   if ((rc = launch_absorb(q_nope, wkv_b, q_lat, B, d_status, stream)) != MLA_OK) return rc;
   if ((rc = launch_attend(q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, scale, o_part, lse_part, B, K, S_max,
-                          n_split, span, d_status, stream)) != MLA_OK)
+                          n_split, span, d_status, stream, true)) != MLA_OK)
     return rc;
-  return launch_combine(o_part, lse_part, wkv_b, out, lse_out, B, n_split, d_status, stream);
+  return launch_combine(o_part, lse_part, wkv_b, out, lse_out, B, n_split, d_status, stream, true);
 }
 
 #ifdef MLA_TRACE

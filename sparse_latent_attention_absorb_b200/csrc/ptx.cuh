@@ -40,6 +40,14 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Programmatic dependent launch.  grid_dep_wait(): block until the grid this
+// one depends on has finished and its memory is visible (a no-op when the
+// launch had no programmatic dependency).  grid_dep_launch(): let the
+// dependent grid start launching once every CTA of this grid has said so or
+// exited.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ----------------------------------------------------------------------------
 // mbarrier
 

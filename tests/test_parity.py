@@ -111,6 +111,45 @@ def test_split_outputs_combine_to_oracle_mix(name):
     assert np.max(np.abs(merged - ref.o_lat)) <= 1e-2 * np.max(np.abs(ref.o_lat)) + 1e-4
 
 
+def test_single_split_attend_writes_the_mixed_latent():
+    """Steps a2-a5 when every row is one split (B > SMs / 2): the attention
+    step's output is the mixed latent O~ itself, in bf16, plus its lse."""
+    name = "small_b80_ctx700_top300"
+    d = wl.generate(name)
+    B, K = d["topk_idx"].shape
+    assert pkg.num_splits(B, K) == 1
+    g = to_dev(d)
+    q_lat = pkg.mla_absorb_q(g["q_nope"], g["wkv_b"])
+    o_lat, lse_part = pkg.mla_sparse_attend(q_lat, g["q_pe"], g["kv_cache"], g["pe_cache"], g["end_pos"],
+                                            g["topk_idx"], g["scale"])
+    torch.cuda.synchronize()
+    assert o_lat.dtype == torch.bfloat16 and tuple(o_lat.shape) == (B, 128, 512)
+    rows = [0, 13, 41, 79]
+    ref = run_oracle(d, rows=rows, want_o_lat=True)
+    got = o_lat.double().cpu().numpy()[rows]
+    assert np.max(np.abs(got - ref.o_lat)) <= 1e-2 * np.max(np.abs(ref.o_lat)) + 1e-4
+    assert np.max(np.abs(lse_part.double().cpu().numpy()[rows, 0] - ref.lse)) <= 1e-2
+
+
+@pytest.mark.parametrize("B", [7, 70])
+def test_combine_step_single_split(B):
+    """Steps a6-a7 with one split: O~ arrives in bf16 and goes straight into
+    the W_UV product; lse passes through.  B = 70 spans two row tiles, the
+    second one ragged."""
+    gen = torch.Generator().manual_seed(11 + B)
+    o_lat = (torch.randn((B, 128, 512), generator=gen) * 0.05).to(torch.bfloat16)
+    lse_part = torch.randn((B, 1, 128), generator=gen, dtype=torch.float32) * 3
+    wkv_b = (torch.randn((128 * 256, 512), generator=gen) * 512 ** -0.5).to(torch.bfloat16)
+    lse_out = torch.empty((B, 128), dtype=torch.float32, device=DEV)
+    out = pkg.mla_combine_value_up(o_lat.to(DEV), lse_part.to(DEV), wkv_b.to(DEV), lse_out=lse_out)
+    torch.cuda.synchronize()
+    w_uv = wkv_b.double().view(128, 256, 512)[:, 128:, :]
+    ref = torch.einsum("bhc,hec->bhe", o_lat.double(), w_uv).numpy()
+    got = out.double().cpu().numpy()
+    assert np.max(np.abs(got - ref)) <= out_bound(ref)
+    assert np.array_equal(lse_out.cpu().numpy(), lse_part[:, 0].numpy())
+
+
 def test_combine_step_with_given_partials():
     """Steps a6-a7 alone on synthetic partials: exact LSE weights, then the
     W_UV product of the bf16-rounded mix."""
