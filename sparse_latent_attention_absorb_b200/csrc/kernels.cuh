@@ -139,9 +139,8 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 //
 // One 2-CTA cluster per (batch row b, key split s).  CTA rank r owns latent
 // columns [256r, 256r+256) and rotary columns [32r, 32r+32) of the score:
-//   * its half of the absorbed query is the A operand of QK: latent columns
-//     0..127 of the half in TMEM (bf16 pairs), columns 128..255 and the
-//     rotary part in shared memory;
+//   * its half of the absorbed query is the A operand of QK: the 256 latent
+//     columns in TMEM (bf16 pairs), the 32 rotary columns in shared memory;
 //   * for every selected position t of the split, a gather warp copies
 //     kv[b,t,its 256] (128B-swizzled rows) and pe[b,t,its 32] (64B-swizzled
 //     rows) into a ring of 64-position tiles (cp.async, 16 bytes per lane);
@@ -151,8 +150,8 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 //     N = 64 positions, into a TMEM score buffer;
 //   * two groups of four softmax warps take alternate tiles.  A thread owns
 //     one head (TMEM lane) and all 64 positions of its group's tiles: it
-//     reads its partial scores (which frees the buffer for the QK two tiles
-//     ahead), rounds them to fp16 in log2 units, pushes them into the peer
+//     reads its partial scores (which frees the one score buffer for the next
+//     tile's QK), rounds them to fp16 in log2 units, pushes them into the peer
 //     CTA's shared memory (st.async, completing on the peer's mbarrier),
 //     adds the peer's half -- both CTAs add the same two fp16 values, so their
 //     scores and everything after are bitwise identical -- masks, takes the
@@ -173,8 +172,7 @@ constexpr int kNt = 64;                            // positions per tile
 constexpr int kStages = 4;                         // gathered tile ring
 constexpr int kLatBlock = kNt * 128;               // one 64-column latent block of a tile (8 KB)
 constexpr int kStageBytes = 4 * kLatBlock + kNt * 64;  // 4 latent blocks + the rotary block: 36 KB
-constexpr int kQsBytes = 2 * kH * 128;             // latent query columns 128..255 of the half: 32 KB
-constexpr int kQpeBytes = kH * 64;                 // 8 KB
+constexpr int kQpeBytes = kH * 64;                 // rotary query columns of the half: 8 KB
 constexpr int kXHalves = (kNt / 8) * kH * 16;      // 16 KB: one exchanged score tile (fp16)
 constexpr int kXBytes = kXHalves + kH * 4;         // + each row's fp32 offset
 constexpr int kMslotBytes = 2 * kH * 4;            // running maximum published by each group
@@ -182,8 +180,7 @@ constexpr int kRedBytes = 4 * kH * 4;              // (row sum, maximum) of each
 constexpr int kBarBytes = 512;
 constexpr int kOffStage = 0;
 constexpr int kOffX = kOffStage + kStages * kStageBytes;
-constexpr int kOffQs = kOffX + 2 * kXBytes;
-constexpr int kOffQpe = kOffQs + kQsBytes;
+constexpr int kOffQpe = kOffX + 2 * kXBytes;
 constexpr int kOffMslot = kOffQpe + kQpeBytes;
 constexpr int kOffRed = kOffMslot + kMslotBytes;
 constexpr int kOffBar = kOffRed + kRedBytes;
@@ -196,17 +193,16 @@ constexpr int kGatherWarps = kStages;  // gather warp g always fills stage g
 // SM sub-partitions, 16K registers each, one of which holds four warps).
 constexpr int kAttendThreads = 32 * (kGatherWarp0 + kGatherWarps);  // 416
 // TMEM columns
-constexpr uint32_t kColS = 0;     // score buffer of group g at kColS + 64g (f32)
-constexpr uint32_t kColP = 128;   // P buffer of group g at kColP + 32g (bf16 pairs)
-constexpr uint32_t kColQ = 192;   // 64 columns: latent query columns 0..127 of the half (bf16 pairs)
+constexpr uint32_t kColS = 0;     // the score buffer (f32)
+constexpr uint32_t kColP = 64;    // P buffer of group g at kColP + 32g (bf16 pairs)
+constexpr uint32_t kColQ = 128;   // 128 columns: the latent query half (bf16 pairs)
 constexpr uint32_t kColO = 256;   // 256 f32 columns of O
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-static_assert(kStageBytes % 1024 == 0 && kOffX % 1024 == 0 && kOffQs % 1024 == 0 && kOffQpe % 1024 == 0 &&
-                  kXBytes % 16 == 0,
+static_assert(kStageBytes % 1024 == 0 && kOffX % 1024 == 0 && kOffQpe % 1024 == 0 && kXBytes % 16 == 0,
               "swizzle atoms");
 static_assert(kAttendSmemBytes <= 232448, "shared memory");
-static_assert(kColS + 2 * kNt <= kColP && kColP + kNt <= kColQ && kColQ + 64 <= kColO, "TMEM map");
+static_assert(kColS + kNt <= kColP && kColP + kNt <= kColQ && kColQ + 128 <= kColO, "TMEM map");
 // Each gather warp owns one stage (tiles g, g+kStages, ...), so every wait on
 // a stage's kv_empty barrier is exactly one phase after the warp's previous
 // wait on it; with fewer stages than warps a waiter could run two phases
@@ -218,8 +214,8 @@ struct AttendBars {
   uint64_t q_full;              // softmax warps (8 arrivals) after storing Q
   uint64_t kv_full[kStages];    // the tile's gather warp (1 arrival) once its copies landed
   uint64_t kv_empty[kStages];   // MMA commit after PV of the tile
-  uint64_t s_full[2];           // MMA commit after QK: partial scores in buffer g
-  uint64_t s_empty[2];          // group g (4 arrivals) after reading its partial scores
+  uint64_t s_full[2];           // MMA commit after QK of a tile of group g: partial scores ready
+  uint64_t s_empty;             // the tile's group (4 arrivals) after reading the partial scores
   uint64_t p_full[2];           // group g (4 arrivals) after writing P
   uint64_t p_free[2];           // MMA commit after PV of the tile: P buffer free, O stable
   uint64_t x_full[2];           // 1 local arrival + kXBytes of the peer group's st.async
@@ -310,7 +306,6 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
 
   const uint32_t sStage = smem_u32(smem + kOffStage);
   const uint32_t sX = smem_u32(smem + kOffX);
-  const uint32_t sQs = smem_u32(smem + kOffQs);
   const uint32_t sQpe = smem_u32(smem + kOffQpe);
   float* mslot = reinterpret_cast<float*>(smem + kOffMslot);  // [group][head]
   float* red = reinterpret_cast<float*>(smem + kOffRed);      // [l | m][group][head]
@@ -327,7 +322,6 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars->s_full[i]), 1);
-      mbar_init(smem_u32(&bars->s_empty[i]), 4);
       mbar_init(smem_u32(&bars->p_full[i]), 4);
       mbar_init(smem_u32(&bars->p_free[i]), 1);
       mbar_init(smem_u32(&bars->x_full[i]), 1);
@@ -335,6 +329,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       mbar_init(smem_u32(&bars->x_free[i]), 4);
       for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&bars->m_ready[i][q]), 1);
     }
+    mbar_init(smem_u32(&bars->s_empty), 4);
     fence_mbarrier_init_cluster();
   }
   if (warp == kMmaWarp) {
@@ -431,7 +426,8 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     // A polling scheduler: PV(pv) as soon as P is written, QK(qk) as soon as
-    // its rows have landed and its score buffer has been read, PV first.
+    // its rows have landed and the previous tile's scores have been read,
+    // PV first.
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kNt, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
@@ -439,17 +435,21 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       // is the base descriptor plus x/16 (start-address field).
       const uint64_t d_lat = smem_desc_sw128(sStage, 16, 1024);            // QK B, latent, K-major
       const uint64_t d_pe = smem_desc_sw64(sStage + 4 * kLatBlock, 512);    // QK B, rotary, K-major
-      const uint64_t d_qs = smem_desc_sw128(sQs, 16, 1024);                 // QK A, latent 128..255, K-major
       const uint64_t d_qpe = smem_desc_sw64(sQpe, 512);                     // QK A, rotary, K-major
       const uint64_t d_v = smem_desc_sw128(sStage, kLatBlock, 1024);        // PV B, latent, N-major
       wait(smem_u32(&bars->q_full), 0, ab);
       tc_fence_after();
       int qk = 0, pv = 0, st_qk = 0, st_pv = 0;
+      // Conditions already seen true are remembered: under load every
+      // mbarrier probe costs a few hundred cycles, so each round tests only
+      // what is still outstanding.
+      bool pv_ok = false, kv_ok = false, se_ok = false;
       uint32_t idle = 0;
       uint64_t idle_since = 0;
       while (pv < n_tiles) {
         bool did = false;
-        if (pv < qk && mbar_test(smem_u32(&bars->p_full[pv & 1]), (pv >> 1) & 1)) {
+        if (pv < qk && !pv_ok) pv_ok = mbar_test(smem_u32(&bars->p_full[pv & 1]), (pv >> 1) & 1);
+        if (pv_ok) {
           tc_fence_after();
           MLA_TRACE_STAMP(kTrPvStart, pv);
           const uint64_t dv = d_v + (uint64_t)((st_pv * kStageBytes) >> 4);
@@ -463,30 +463,31 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
           MLA_TRACE_STAMP(kTrPvIssued, pv);
           ++pv;
           st_pv = (st_pv + 1 == kStages) ? 0 : st_pv + 1;
+          pv_ok = false;
           did = true;
-        } else if (qk < n_tiles && mbar_test(smem_u32(&bars->kv_full[st_qk]), (qk / kStages) & 1) &&
-                   (qk < 2 || mbar_test(smem_u32(&bars->s_empty[qk & 1]), ((qk >> 1) - 1) & 1))) {
-          tc_fence_after();
-          MLA_TRACE_STAMP(kTrQkStart, qk);
-          const uint64_t dl = d_lat + (uint64_t)((st_qk * kStageBytes) >> 4);
-          const uint64_t dr = d_pe + (uint64_t)((st_qk * kStageBytes) >> 4);
-          const uint32_t dst = tmem + kColS + (qk & 1) * kNt;
+        } else if (qk < n_tiles) {
+          if (!kv_ok) kv_ok = mbar_test(smem_u32(&bars->kv_full[st_qk]), (qk / kStages) & 1);
+          if (kv_ok && !se_ok) se_ok = qk == 0 || mbar_test(smem_u32(&bars->s_empty), (qk - 1) & 1);
+          if (se_ok) {
+            tc_fence_after();
+            MLA_TRACE_STAMP(kTrQkStart, qk);
+            const uint64_t dl = d_lat + (uint64_t)((st_qk * kStageBytes) >> 4);
+            const uint64_t dr = d_pe + (uint64_t)((st_qk * kStageBytes) >> 4);
+            const uint32_t dst = tmem + kColS;
 #pragma unroll
-          for (int k = 0; k < 8; ++k)  // latent 0..127: A from TMEM
-            mma_ts(dst, tmem + kColQ + k * 8, dl + (uint64_t)(((k >> 2) * kLatBlock + (k & 3) * 32) >> 4), idesc_qk,
-                   k > 0 ? 1u : 0u);
+            for (int k = 0; k < 16; ++k)  // latent: A from TMEM
+              mma_ts(dst, tmem + kColQ + k * 8, dl + (uint64_t)(((k >> 2) * kLatBlock + (k & 3) * 32) >> 4),
+                     idesc_qk, k > 0 ? 1u : 0u);
 #pragma unroll
-          for (int k = 8; k < 16; ++k)  // latent 128..255: A from shared memory
-            mma_ss(dst, d_qs + (uint64_t)((((k - 8) >> 2) * (kH * 128) + (k & 3) * 32) >> 4),
-                   dl + (uint64_t)(((k >> 2) * kLatBlock + (k & 3) * 32) >> 4), idesc_qk, 1u);
-#pragma unroll
-          for (int k = 0; k < 2; ++k)  // rotary: 32 bytes per step inside the 64-byte rows
-            mma_ss(dst, d_qpe + (uint64_t)((k * 32) >> 4), dr + (uint64_t)((k * 32) >> 4), idesc_qk, 1u);
-          mma_commit(smem_u32(&bars->s_full[qk & 1]));
-          MLA_TRACE_STAMP(kTrQkIssued, qk);
-          ++qk;
-          st_qk = (st_qk + 1 == kStages) ? 0 : st_qk + 1;
-          did = true;
+            for (int k = 0; k < 2; ++k)  // rotary: 32 bytes per step inside the 64-byte rows
+              mma_ss(dst, d_qpe + (uint64_t)((k * 32) >> 4), dr + (uint64_t)((k * 32) >> 4), idesc_qk, 1u);
+            mma_commit(smem_u32(&bars->s_full[qk & 1]));
+            MLA_TRACE_STAMP(kTrQkIssued, qk);
+            ++qk;
+            st_qk = (st_qk + 1 == kStages) ? 0 : st_qk + 1;
+            kv_ok = se_ok = false;
+            did = true;
+          }
         }
         if (did) {
           idle = 0;
@@ -514,38 +515,25 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     const bool leader = (qd == 0 && lane == 0);
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
 
-    // This CTA's half of the query: latent columns 0..127 into TMEM (group
-    // 0), latent columns 128..255 into shared memory as two 128B-swizzled
-    // K-major blocks and the 32 rotary values as a 64B-swizzled K-major row
-    // (group 1).
+    // This CTA's half of the query: latent columns 0..127 (group 0) and
+    // 128..255 (group 1) into TMEM; the 32 rotary values (group 1) into shared
+    // memory as a 64B-swizzled K-major row.
     {
       grid_dep_wait();  // q_lat comes from the absorption kernel
       const uint4* ql = reinterpret_cast<const uint4*>(q_lat + ((size_t)b * kH + i) * kDl + rank * 256);
-      if (grp == 0) {
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {  // 64 latent values = 32 columns each
-          uint32_t r[32];
+      for (int part = 0; part < 2; ++part) {  // 64 latent values = 32 columns each
+        uint32_t r[32];
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const uint4 x = __ldg(ql + part * 8 + v);
-            r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
-          }
-          tmem_st32(tmem + lane_base + kColQ + part * 32, r);
+        for (int v = 0; v < 8; ++v) {
+          const uint4 x = __ldg(ql + (2 * grp + part) * 8 + v);
+          r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
         }
-        tmem_wait_st();
-        tc_fence_before();
-      } else {
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const uint4 x = __ldg(ql + (2 + part) * 8 + v);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sQs + part * (kH * 128) +
-                                                                          sw128_offset(i, v)),
-                         "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w)
-                         : "memory");
-          }
-        }
+        tmem_st32(tmem + lane_base + kColQ + (2 * grp + part) * 32, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      if (grp == 1) {
         const uint4* qp = reinterpret_cast<const uint4*>(q_pe + ((size_t)b * kH + i) * kDr + rank * 32);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -560,7 +548,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));
     }
 
-    const uint32_t sbuf = tmem + lane_base + kColS + grp * kNt;
+    const uint32_t sbuf = tmem + lane_base + kColS;
     const uint32_t pbuf = tmem + lane_base + kColP + grp * (kNt / 2);
     const uint32_t x_mine = sX + grp * kXBytes;              // the peer's half arrives here
     const uint32_t x_peer = cluster_map(x_mine, peer);       // our half goes there
@@ -593,7 +581,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[grp]));
+        if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty));
         float om = __uint_as_float(sv[0]);
 #pragma unroll
         for (int t = 1; t < 64; ++t) om = fmaxf(om, __uint_as_float(sv[t]));

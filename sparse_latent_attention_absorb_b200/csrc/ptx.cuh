@@ -199,6 +199,21 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t a, ui
                : "memory");
 }
 
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into a
+// cluster peer's, completing `bytes` transactions on the peer's mbarrier.
+// Runs on the copy engine: one instruction instead of per-lane stores.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
+                                                  uint32_t remote_bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst_cluster),
+               "r"(src_cta), "r"(bytes), "r"(remote_bar)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until this thread's committed bulk copies have finished reading their
+// sources (the source buffers may then be overwritten).
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
 __device__ __forceinline__ void st_async_b32(uint32_t remote_addr, uint32_t a, uint32_t remote_bar) {
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote_addr), "r"(a),
                "r"(remote_bar)
