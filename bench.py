@@ -188,7 +188,9 @@ def gpu_arm(args, rank, world, device):
         if rc != 0:
             raise binding.MLAError(rc, "mla_sparse_decode")
 
-    # one CUDA graph per input set: a replay is exactly one decode call
+    # One CUDA graph per input set (a replay is exactly one decode call), and
+    # one graph of NSETS consecutive calls, one per set, so that steps timed
+    # back to back do not each pay a graph launch.
     with torch.cuda.stream(stream):
         for i in range(len(sets)):
             call(i, stream)
@@ -199,7 +201,18 @@ def gpu_arm(args, rank, world, device):
         with torch.cuda.graph(g, stream=stream):
             call(i, torch.cuda.current_stream())
         graphs.append(g)
+    chain = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(chain, stream=stream):
+        for i in range(len(sets)):
+            call(i, torch.cuda.current_stream())
     torch.cuda.synchronize()
+
+    def run_steps(n):
+        """n decode steps, input sets in rotation (n // NSETS chain replays, then singles)."""
+        for _ in range(n // NSETS):
+            chain.replay()
+        for i in range(n % NSETS):
+            graphs[i].replay()
 
     def barrier():
         if world > 1:
@@ -207,8 +220,7 @@ def gpu_arm(args, rank, world, device):
 
     # ---- timed region: K decode steps
     with torch.cuda.stream(stream):
-        for it in range(args.warmup):
-            graphs[it % NSETS].replay()
+        run_steps(args.warmup)
     stream.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -216,8 +228,7 @@ def gpu_arm(args, rank, world, device):
     with ClockSampler(torch.cuda.current_device() if device.index is None else device.index) as clocks:
         with torch.cuda.stream(stream):
             ev0.record(stream)
-            for it in range(args.steps):
-                graphs[it % NSETS].replay()
+            run_steps(args.steps)
             ev1.record(stream)
         stream.synchronize()
     barrier()
@@ -253,15 +264,24 @@ def gpu_arm(args, rank, world, device):
         return lib.mla_combine_value_up(P(o_part), P(lse_part), P(sets[i]["wkv_b"]), P(outs[i]), None, B, n_split, sv)
 
     def time_kernel(fn, reps):
+        """Device time of one launch: `reps` back-to-back launches (input sets
+        rotating) captured in a CUDA graph, so host launch cost is excluded."""
         with torch.cuda.stream(stream):
             for r in range(4):
                 assert fn(r % NSETS) == 0
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
             for r in range(reps):
                 fn(r % NSETS)
+        with torch.cuda.stream(stream):
+            g.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
             e1.record(stream)
         stream.synchronize()
+        del g
         return e0.elapsed_time(e1) / reps
 
     with torch.cuda.stream(stream):
@@ -334,7 +354,7 @@ def gpu_arm(args, rank, world, device):
                    "parallelism": f"replicas x{world} (batch rows)",
                    "l2": f"{NSETS} rotating input sets (queries, indices, wkv_b copy each); per-step footprint "
                          f"{call_bytes / 1e6:.0f} MB > 126 MB L2",
-                   "timing": "CUDA graph replay per step, CUDA events on the launching stream"},
+                   "timing": "CUDA graphs of 4 consecutive steps (one per input set), CUDA events on the launching stream"},
         "roofline": {"bound": "hbm", "kernel": "sparse_attend_kernel", "achieved": achieved, "peak": hbm,
                      "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
                      "peak_source": f"{kind} hbm_gbs", "alg_bytes_per_launch": a_bytes,

@@ -38,48 +38,51 @@ __device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* p) {
 // =============================================================================
 // absorb_kernel: q_lat[b,h,c] = sum_d q_nope[b,h,d] * W_UK[h,d,c]
 //
-// Swap-AB GEMM per (head h, 128-column chunk of c, tile of up to 128 rows b):
-//   D[c, b] = sum_d W_UK[h, d, c] * q_nope[b, h, d]
-// M = 128 (c), N = batch tile (multiple of 16), K = 128 (d).
-// A = W_UK[h][:, chunk] is M-major in memory (c contiguous): two TMA boxes of
-// 64 c x 128 d, 128B-swizzled.  B = q_nope[:, h, :] is K-major: two 3-D TMA
-// boxes of 64 d x N rows.  The accumulator lives in TMEM (lanes = c).
+// Per (latent half, head h, tile of up to 128 rows b):
+//   D[b, c] = sum_d q_nope[b, h, d] * W_UK[h, d, c]
+// M = 128 (rows b; rows past B are zero-filled by TMA), N = 256 (the half's
+// latent columns c, two MMAs of N = 128), K = 128 (d).  A = q_nope[:, h, :] is
+// K-major (two 3-D TMA boxes of 64 d x 128 rows); B = W_UK[h][:, half] is
+// N-major (c contiguous): four TMA boxes of 64 c x 128 d.  The two N = 128
+// quarters have their own barriers, so the first MMA starts while the second
+// quarter is still landing, and the first quarter's epilogue overlaps the
+// second MMA.  Epilogue: TMEM lane = row b, so each thread writes its row's
+// 128 columns of a quarter as 16-byte stores.
 // =============================================================================
-constexpr int kAbsorbNMax = 128;
-constexpr int kAbsorbSmemA = 2 * 64 * 128 * 2;                      // 32 KB
-// shared memory for a batch tile of n rows: W_UK chunk, q_nope tile, barriers
-// (sized to the tile so that four CTAs fit on an SM when n <= 64)
-__host__ __device__ constexpr int absorb_smem_bytes(int n) { return kAbsorbSmemA + 2 * n * 128 + 256 + kSmemAlignPad; }
-constexpr int kAbsorbSmemBytes = absorb_smem_bytes(kAbsorbNMax);
+constexpr int kAbsorbRows = 128;
+constexpr int kAbsorbSmemA = 2 * kAbsorbRows * 128;                  // q_nope tile: 32 KB
+constexpr int kAbsorbSmemB = 4 * 64 * 128 * 2;                       // W_UK half: 64 KB
+constexpr int kAbsorbSmemBytes = kAbsorbSmemA + kAbsorbSmemB + 256 + kSmemAlignPad;  // + barriers
 
 __global__ void __launch_bounds__(128, 1)
 absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
-              __nv_bfloat16* __restrict__ q_lat, int B, int n_tile, int* d_status) {
+              __nv_bfloat16* __restrict__ q_lat, int B, int* d_status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int chunk = blockIdx.x;  // 128-wide chunk of the latent dimension
+  const int half = blockIdx.x;  // latent columns [256 half, 256 half + 256)
   const int h = blockIdx.y;
-  const int b0 = blockIdx.z * kAbsorbNMax;
+  const int b0 = blockIdx.z * kAbsorbRows;
 
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + kAbsorbSmemA;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAbsorbSmemA + 2 * n_tile * 128);
-  const uint32_t bar_load = smem_u32(&bars[0]);
-  const uint32_t bar_mma = smem_u32(&bars[1]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[3]);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAbsorbSmemA + kAbsorbSmemB);
+  const uint32_t bar_load[2] = {smem_u32(&bars[0]), smem_u32(&bars[1])};
+  const uint32_t bar_mma[2] = {smem_u32(&bars[2]), smem_u32(&bars[3])};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[4]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[5]);
   const AbortState ab{abort_flag, d_status};
 
-  const uint32_t tmem_cols = n_tile <= 32 ? 32u : (n_tile <= 64 ? 64u : 128u);
   if (tid == 0) {
     *abort_flag = 0;
-    mbar_init(bar_load, 1);
-    mbar_init(bar_mma, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_load[i], 1);
+      mbar_init(bar_mma[i], 1);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), tmem_cols);
+    tmem_alloc(smem_u32(tmem_slot), 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -90,48 +93,58 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
   if (tid == 0) {
     tma_prefetch_desc(&tm_w);
     tma_prefetch_desc(&tm_q);
-    mbar_arrive_expect_tx(bar_load, kAbsorbSmemA + 2 * n_tile * 128);
     const int wrow = h * kHeadRows;  // W_UK rows of head h
-    tma_load_2d(sA, &tm_w, bar_load, chunk * 128, wrow);
-    tma_load_2d(sA + 64 * 128 * 2, &tm_w, bar_load, chunk * 128 + 64, wrow);
-    tma_load_3d(sB, &tm_q, bar_load, 0, h, b0);
-    tma_load_3d(sB + n_tile * 128, &tm_q, bar_load, 64, h, b0);
+    // quarter 0: the query tile and the first two W boxes; quarter 1: the other two
+    mbar_arrive_expect_tx(bar_load[0], kAbsorbSmemA + 2 * 64 * 128 * 2);
+    tma_load_3d(sA, &tm_q, bar_load[0], 0, h, b0);
+    tma_load_3d(sA + kAbsorbRows * 128, &tm_q, bar_load[0], 64, h, b0);
+    mbar_arrive_expect_tx(bar_load[1], 2 * 64 * 128 * 2);
+    for (int box = 0; box < 4; ++box)
+      tma_load_2d(sB + box * (64 * 128 * 2), &tm_w, bar_load[box >> 1], half * 256 + box * 64, wrow);
     grid_dep_launch();  // the attention kernel may start gathering
 
-    wait(bar_load, 0, ab);
-    tc_fence_after();
-    const uint32_t idesc = idesc_bf16_f32(128, n_tile, /*a MN*/ true, /*b MN*/ false);
-    for (int k = 0; k < kDn / 16; ++k) {
-      // A: 16 d-rows per step (two 8-row groups 1024 B apart); the two
-      // 64-wide c blocks are 16 KB apart.
-      const uint64_t a = smem_desc_sw128(sA + k * 16 * 128, 64 * 128 * 2, 1024);
-      // B: 32 bytes of d per step inside the 128-byte row; the second
-      // 64-wide d block follows the first.
-      const uint64_t b = smem_desc_sw128(sB + (k >> 2) * n_tile * 128 + (k & 3) * 32, 16, 1024);
-      mma_ss(tmem, a, b, idesc, k > 0 ? 1u : 0u);
+    constexpr uint32_t idesc = idesc_bf16_f32(128, 128, /*a MN*/ false, /*b MN*/ true);
+    for (int qtr = 0; qtr < 2; ++qtr) {
+      wait(bar_load[qtr], 0, ab);
+      tc_fence_after();
+      for (int k = 0; k < kDn / 16; ++k) {
+        // A: 32 bytes of d per step inside the 128-byte rows; the second
+        // 64-wide d block follows the first.
+        const uint64_t a = smem_desc_sw128(sA + (k >> 2) * (kAbsorbRows * 128) + (k & 3) * 32, 16, 1024);
+        // B: 16 d-rows per step (two 8-row groups 1024 B apart); the two
+        // 64-wide c blocks of the quarter are 16 KB apart.
+        const uint64_t bd = smem_desc_sw128(sB + qtr * (2 * 64 * 128 * 2) + k * 16 * 128, 64 * 128 * 2, 1024);
+        mma_ss(tmem + qtr * 128, a, bd, idesc, k > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_mma[qtr]);
     }
-    mma_commit(bar_mma);
   }
   __syncwarp();
 
-  // Epilogue: lane (32*warp + lane) holds column c of the chunk, one TMEM
-  // column per batch row.
-  wait(bar_mma, 0, ab);
-  tc_fence_after();
-  const int c = chunk * 128 + warp * 32 + lane;
-  for (int n0 = 0; n0 < n_tile; n0 += 16) {
-    uint32_t v[16];
-    tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + n0, v);
-    tmem_wait_ld();
+  // Epilogue: lane (32*warp + lane) holds row b, 128 f32 columns per quarter.
+  const int b = b0 + warp * 32 + lane;
+  for (int qtr = 0; qtr < 2; ++qtr) {
+    wait(bar_mma[qtr], 0, ab);
+    tc_fence_after();
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t v[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + qtr * 128 + cc * 32, v);
+      tmem_wait_ld();
+      if (b < B) {
+        uint4* dst = reinterpret_cast<uint4*>(q_lat + ((size_t)b * kH + h) * kDl + half * 256 + qtr * 128 + cc * 32);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int b = b0 + n0 + j;
-      if (b < B) q_lat[((size_t)b * kH + h) * kDl + c] = __float2bfloat16_rn(__uint_as_float(v[j]));
+        for (int t = 0; t < 4; ++t)
+          dst[t] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * t]), __uint_as_float(v[8 * t + 1])),
+                              pack_bf16x2(__uint_as_float(v[8 * t + 2]), __uint_as_float(v[8 * t + 3])),
+                              pack_bf16x2(__uint_as_float(v[8 * t + 4]), __uint_as_float(v[8 * t + 5])),
+                              pack_bf16x2(__uint_as_float(v[8 * t + 6]), __uint_as_float(v[8 * t + 7])));
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, tmem_cols);
+  if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 // =============================================================================
@@ -164,9 +177,13 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 // The split's normalised O and its log-sum-exp go to o_part / lse_part (O in
 // f32 per split; with a single split per row, the final O~ in bf16).
 //
-// Warp roles (416 threads): warps 0-3 softmax group 0 (even tiles), warps
+// Warp roles (448 threads): warps 0-3 softmax group 0 (even tiles), warps
 // 4-7 softmax group 1 (odd tiles), warp w covering TMEM lanes 32(w%4)..;
-// warp 8 TMEM allocation + MMA issue; warps 9-12 gather (one stage each).
+// warp 8 TMEM allocation + QK issue; warp 9 PV issue; warps 10-13 gather (one
+// stage each).  QK and PV are issued by different threads: their MMAs
+// interleave in the tensor pipe, and a commit (which tracks the issuing
+// thread's MMAs only) signals PV completion without waiting for a QK queued
+// ahead of it.
 // =============================================================================
 constexpr int kNt = 64;                            // positions per tile
 constexpr int kStages = 4;                         // gathered tile ring
@@ -186,12 +203,13 @@ constexpr int kOffRed = kOffMslot + kMslotBytes;
 constexpr int kOffBar = kOffRed + kRedBytes;
 constexpr int kAttendSmemBytes = kOffBar + kBarBytes + kSmemAlignPad;
 constexpr int kSoftmaxWarps = 8;                   // two groups of four
-constexpr int kMmaWarp = 8;
-constexpr int kGatherWarp0 = 9;
+constexpr int kMmaWarp = 8;     // TMEM allocation, QK issue
+constexpr int kPvWarp = 9;      // PV issue
+constexpr int kGatherWarp0 = 10;
 constexpr int kGatherWarps = kStages;  // gather warp g always fills stage g
-// 13 warps: at most 128 registers a thread (the warps spread over the four
-// SM sub-partitions, 16K registers each, one of which holds four warps).
-constexpr int kAttendThreads = 32 * (kGatherWarp0 + kGatherWarps);  // 416
+// 14 warps: at most 128 registers a thread (the warps spread over the four
+// SM sub-partitions, 16K registers each, two of which hold four warps).
+constexpr int kAttendThreads = 32 * (kGatherWarp0 + kGatherWarps);  // 448
 // TMEM columns
 constexpr uint32_t kColS = 0;     // the score buffer (f32)
 constexpr uint32_t kColP = 64;    // P buffer of group g at kColP + 32g (bf16 pairs)
@@ -208,7 +226,7 @@ static_assert(kColS + kNt <= kColP && kColP + kNt <= kColQ && kColQ + 128 <= kCo
 // wait on it; with fewer stages than warps a waiter could run two phases
 // ahead of the barrier, where a parity test cannot tell the phases apart.
 static_assert(kGatherWarps == kStages, "one stage per gather warp");
-static_assert(kMmaWarp == kSoftmaxWarps && kGatherWarp0 == kMmaWarp + 1, "warp roles");
+static_assert(kMmaWarp == kSoftmaxWarps && kPvWarp == kMmaWarp + 1 && kGatherWarp0 == kPvWarp + 1, "warp roles");
 
 struct AttendBars {
   uint64_t q_full;              // softmax warps (8 arrivals) after storing Q
@@ -272,6 +290,7 @@ enum TraceEvent {
 constexpr int kTraceTiles = 512;
 #ifdef MLA_TRACE
 __device__ long long g_mla_trace[2 * kTrEvents * kTraceTiles];
+__device__ unsigned long long g_mla_cluster_ns[2 * 4096];  // per cluster: start, end (globaltimer)
 #define MLA_TRACE_STAMP(ev, tile)                                                               \
   do {                                                                                           \
     if ((blockIdx.x >> 1) == 0 && (tile) < kTraceTiles)                                          \
@@ -341,6 +360,9 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
   tc_fence_after();
   const uint32_t tmem = bars->tmem_addr;
   grid_dep_launch();  // the combine kernel may start loading its weights
+#ifdef MLA_TRACE
+  if (rank == 0 && tid == 0 && unit < 4096) g_mla_cluster_ns[2 * unit] = global_timer_ns();
+#endif
 
   if (warp >= kGatherWarp0) {
     // ------------------------------------------------------------ gather
@@ -424,86 +446,57 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       }
     }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issue
-    // A polling scheduler: PV(pv) as soon as P is written, QK(qk) as soon as
-    // its rows have landed and the previous tile's scores have been read,
-    // PV first.
+    // ------------------------------------------------------------ QK issue
+    // QK(j) as soon as its rows have landed and the previous tile's scores
+    // have been read (one score buffer).
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kNt, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
       // Descriptors are built once; an operand at byte offset x from a base
       // is the base descriptor plus x/16 (start-address field).
       const uint64_t d_lat = smem_desc_sw128(sStage, 16, 1024);            // QK B, latent, K-major
       const uint64_t d_pe = smem_desc_sw64(sStage + 4 * kLatBlock, 512);    // QK B, rotary, K-major
       const uint64_t d_qpe = smem_desc_sw64(sQpe, 512);                     // QK A, rotary, K-major
-      const uint64_t d_v = smem_desc_sw128(sStage, kLatBlock, 1024);        // PV B, latent, N-major
       wait(smem_u32(&bars->q_full), 0, ab);
-      tc_fence_after();
-      int qk = 0, pv = 0, st_qk = 0, st_pv = 0;
-      // Conditions already seen true are remembered: under load every
-      // mbarrier probe costs a few hundred cycles, so each round tests only
-      // what is still outstanding.
-      bool pv_ok = false, kv_ok = false, se_ok = false;
-      uint32_t idle = 0;
-      uint64_t idle_since = 0;
-      while (pv < n_tiles) {
-        bool did = false;
-        if (pv < qk && !pv_ok) pv_ok = mbar_test(smem_u32(&bars->p_full[pv & 1]), (pv >> 1) & 1);
-        if (pv_ok) {
-          tc_fence_after();
-          MLA_TRACE_STAMP(kTrPvStart, pv);
-          const uint64_t dv = d_v + (uint64_t)((st_pv * kStageBytes) >> 4);
-          const uint32_t pa = tmem + kColP + (pv & 1) * (kNt / 2);
+      for (int qk = 0, st = 0; qk < n_tiles; ++qk, st = (st + 1 == kStages) ? 0 : st + 1) {
+        wait(smem_u32(&bars->kv_full[st]), (qk / kStages) & 1, ab);
+        if (qk > 0) wait(smem_u32(&bars->s_empty), (qk - 1) & 1, ab);
+        tc_fence_after();
+        MLA_TRACE_STAMP(kTrQkStart, qk);
+        const uint64_t dl = d_lat + (uint64_t)((st * kStageBytes) >> 4);
+        const uint64_t dr = d_pe + (uint64_t)((st * kStageBytes) >> 4);
+        const uint32_t dst = tmem + kColS;
 #pragma unroll
-          for (int k = 0; k < kNt / 16; ++k)  // 16 positions per step
-            mma_ts(tmem + kColO, pa + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4), idesc_pv,
-                   (pv > 0 || k > 0) ? 1u : 0u);
-          mma_commit(smem_u32(&bars->kv_empty[st_pv]));
-          mma_commit(smem_u32(&bars->p_free[pv & 1]));
-          MLA_TRACE_STAMP(kTrPvIssued, pv);
-          ++pv;
-          st_pv = (st_pv + 1 == kStages) ? 0 : st_pv + 1;
-          pv_ok = false;
-          did = true;
-        } else if (qk < n_tiles) {
-          if (!kv_ok) kv_ok = mbar_test(smem_u32(&bars->kv_full[st_qk]), (qk / kStages) & 1);
-          if (kv_ok && !se_ok) se_ok = qk == 0 || mbar_test(smem_u32(&bars->s_empty), (qk - 1) & 1);
-          if (se_ok) {
-            tc_fence_after();
-            MLA_TRACE_STAMP(kTrQkStart, qk);
-            const uint64_t dl = d_lat + (uint64_t)((st_qk * kStageBytes) >> 4);
-            const uint64_t dr = d_pe + (uint64_t)((st_qk * kStageBytes) >> 4);
-            const uint32_t dst = tmem + kColS;
+        for (int k = 0; k < 16; ++k)  // latent: A from TMEM
+          mma_ts(dst, tmem + kColQ + k * 8, dl + (uint64_t)(((k >> 2) * kLatBlock + (k & 3) * 32) >> 4), idesc_qk,
+                 k > 0 ? 1u : 0u);
 #pragma unroll
-            for (int k = 0; k < 16; ++k)  // latent: A from TMEM
-              mma_ts(dst, tmem + kColQ + k * 8, dl + (uint64_t)(((k >> 2) * kLatBlock + (k & 3) * 32) >> 4),
-                     idesc_qk, k > 0 ? 1u : 0u);
+        for (int k = 0; k < 2; ++k)  // rotary: 32 bytes per step inside the 64-byte rows
+          mma_ss(dst, d_qpe + (uint64_t)((k * 32) >> 4), dr + (uint64_t)((k * 32) >> 4), idesc_qk, 1u);
+        mma_commit(smem_u32(&bars->s_full[qk & 1]));
+        MLA_TRACE_STAMP(kTrQkIssued, qk);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kPvWarp) {
+    // ------------------------------------------------------------ PV issue
+    // PV(j) as soon as its P is written; its commits free the stage and the
+    // P buffer and mark O stable.
+    if (lane == 0 && n_tiles > 0) {
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+      const uint64_t d_v = smem_desc_sw128(sStage, kLatBlock, 1024);  // PV B, latent, N-major
+      for (int pv = 0, st = 0; pv < n_tiles; ++pv, st = (st + 1 == kStages) ? 0 : st + 1) {
+        wait(smem_u32(&bars->p_full[pv & 1]), (pv >> 1) & 1, ab);
+        tc_fence_after();
+        MLA_TRACE_STAMP(kTrPvStart, pv);
+        const uint64_t dv = d_v + (uint64_t)((st * kStageBytes) >> 4);
+        const uint32_t pa = tmem + kColP + (pv & 1) * (kNt / 2);
 #pragma unroll
-            for (int k = 0; k < 2; ++k)  // rotary: 32 bytes per step inside the 64-byte rows
-              mma_ss(dst, d_qpe + (uint64_t)((k * 32) >> 4), dr + (uint64_t)((k * 32) >> 4), idesc_qk, 1u);
-            mma_commit(smem_u32(&bars->s_full[qk & 1]));
-            MLA_TRACE_STAMP(kTrQkIssued, qk);
-            ++qk;
-            st_qk = (st_qk + 1 == kStages) ? 0 : st_qk + 1;
-            kv_ok = se_ok = false;
-            did = true;
-          }
-        }
-        if (did) {
-          idle = 0;
-        } else if (idle++ == 0) {
-          idle_since = global_timer_ns();
-        } else {
-          __nanosleep(40);  // keep the barrier probes from crowding the shared-memory pipe
-        }
-        if (!did && (idle & 255u) == 0 && idle > 0) {
-          if (bars->abort_flag) break;
-          if (global_timer_ns() - idle_since > kWaitLimitNs) {
-            bars->abort_flag = 1;
-            if (d_status) atomicCAS(d_status, 0, MLA_ERR_DEVICE_TIMEOUT);
-            break;
-          }
-        }
+        for (int k = 0; k < kNt / 16; ++k)  // 16 positions per step
+          mma_ts(tmem + kColO, pa + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4), idesc_pv,
+                 (pv > 0 || k > 0) ? 1u : 0u);
+        mma_commit(smem_u32(&bars->kv_empty[st]));
+        mma_commit(smem_u32(&bars->p_free[pv & 1]));
+        MLA_TRACE_STAMP(kTrPvIssued, pv);
       }
     }
     __syncwarp();
@@ -787,6 +780,9 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+#ifdef MLA_TRACE
+  if (rank == 0 && tid == 0 && unit < 4096) g_mla_cluster_ns[2 * unit + 1] = global_timer_ns();
+#endif
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
   cluster_sync();
 }
@@ -808,7 +804,7 @@ constexpr int kCombineMaxSplits = 128;
 constexpr int kCombineSmemA = 8 * 128 * 128;             // 128 KB
 constexpr int kCombineSmemB = 8 * kCombineNMax * 128;    // 64 KB
 constexpr int kCombineSmemCoef = kCombineNMax * kCombineMaxSplits * 4;  // 32 KB
-constexpr int kCombineSmemBytes = kCombineSmemA + kCombineSmemB + kCombineSmemCoef + 256 + kSmemAlignPad;
+constexpr int kCombineSmemBytes = kCombineSmemA + kCombineSmemB + kCombineSmemCoef + 128 + kSmemAlignPad;
 constexpr int kCombineThreads = 256;
 static_assert(kCombineSmemBytes <= 232448, "shared memory");
 
@@ -828,19 +824,18 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
   const uint32_t sB = sA + kCombineSmemA;
   float* coef = reinterpret_cast<float*>(smem + kCombineSmemA + kCombineSmemB);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kCombineSmemA + kCombineSmemB + kCombineSmemCoef);
-  const uint32_t bar_w = smem_u32(&bars[0]);
-  const uint32_t bar_mma = smem_u32(&bars[1]);
-  const uint32_t bar_o = smem_u32(&bars[2]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[3]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[4]);
+  // bar_k[kb]: W_UV box kb (and, with one split, O~ box kb) landed
+  auto bar_k = [&](int kb) { return smem_u32(&bars[kb]); };
+  const uint32_t bar_mma = smem_u32(&bars[8]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[9]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[10]);
   const AbortState ab{abort_flag, d_status};
   const uint32_t tmem_cols = n_tile <= 32 ? 32u : 64u;
 
   if (tid == 0) {
     *abort_flag = 0;
-    mbar_init(bar_w, 1);
+    for (int kb = 0; kb < 8; ++kb) mbar_init(bar_k(kb), 1);
     mbar_init(bar_mma, 1);
-    mbar_init(bar_o, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -854,19 +849,20 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
 
   if (tid == 0) {
     tma_prefetch_desc(&tm_w);
-    mbar_arrive_expect_tx(bar_w, kCombineSmemA);
     const int wrow = h * kHeadRows + kDn;  // W_UV rows of head h
-    for (int kb = 0; kb < 8; ++kb) tma_load_2d(sA + kb * 128 * 128, &tm_w, bar_w, kb * 64, wrow);
+    for (int kb = 0; kb < 8; ++kb) {
+      mbar_arrive_expect_tx(bar_k(kb), 128 * 128 + (n_split == 1 ? n_tile * 128 : 0));
+      tma_load_2d(sA + kb * 128 * 128, &tm_w, bar_k(kb), kb * 64, wrow);
+    }
   }
   grid_dep_wait();  // o_part / lse_part come from the attention kernel
 
   if (n_split == 1) {
     // O~ rows b0.. of head h: eight boxes of 64 columns x n_tile rows (rows
-    // past B read as zero)
+    // past B read as zero), each completing its k-block's barrier
     if (tid == 0) {
       tma_prefetch_desc(&tm_o);
-      mbar_arrive_expect_tx(bar_o, 8 * n_tile * 128);
-      for (int kb = 0; kb < 8; ++kb) tma_load_3d(sB + kb * n_tile * 128, &tm_o, bar_o, kb * 64, h, b0);
+      for (int kb = 0; kb < 8; ++kb) tma_load_3d(sB + kb * n_tile * 128, &tm_o, bar_k(kb), kb * 64, h, b0);
     }
     if (tid < rows && lse_out) lse_out[(size_t)(b0 + tid) * kH + h] = lse_part[(size_t)(b0 + tid) * kH + h];
   } else {
@@ -916,14 +912,15 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
   __syncthreads();
 
   if (tid == 0) {
-    wait(bar_w, 0, ab);
-    if (n_split == 1) wait(bar_o, 0, ab);
-    tc_fence_after();
     const uint32_t idesc = idesc_bf16_f32(128, n_tile, false, false);
-    for (int k = 0; k < kDl / 16; ++k) {
-      const uint64_t a = smem_desc_sw128(sA + (k >> 2) * (128 * 128) + (k & 3) * 32, 16, 1024);
-      const uint64_t bd = smem_desc_sw128(sB + (k >> 2) * (n_tile * 128) + (k & 3) * 32, 16, 1024);
-      mma_ss(tmem, a, bd, idesc, k > 0 ? 1u : 0u);
+    for (int kb = 0; kb < 8; ++kb) {  // each 64-column k-block as soon as it has landed
+      wait(bar_k(kb), 0, ab);
+      tc_fence_after();
+      for (int k = 4 * kb; k < 4 * kb + 4; ++k) {
+        const uint64_t a = smem_desc_sw128(sA + (k >> 2) * (128 * 128) + (k & 3) * 32, 16, 1024);
+        const uint64_t bd = smem_desc_sw128(sB + (k >> 2) * (n_tile * 128) + (k & 3) * 32, 16, 1024);
+        mma_ss(tmem, a, bd, idesc, k > 0 ? 1u : 0u);
+      }
     }
     mma_commit(bar_mma);
   }
