@@ -38,51 +38,56 @@ __device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* p) {
 // =============================================================================
 // absorb_kernel: q_lat[b,h,c] = sum_d q_nope[b,h,d] * W_UK[h,d,c]
 //
-// Per (latent half, head h, tile of up to 128 rows b):
-//   D[b, c] = sum_d q_nope[b, h, d] * W_UK[h, d, c]
-// M = 128 (rows b; rows past B are zero-filled by TMA), N = 256 (the half's
-// latent columns c, two MMAs of N = 128), K = 128 (d).  A = q_nope[:, h, :] is
-// K-major (two 3-D TMA boxes of 64 d x 128 rows); B = W_UK[h][:, half] is
-// N-major (c contiguous): four TMA boxes of 64 c x 128 d.  The two N = 128
-// quarters have their own barriers, so the first MMA starts while the second
-// quarter is still landing, and the first quarter's epilogue overlaps the
-// second MMA.  Epilogue: TMEM lane = row b, so each thread writes its row's
-// 128 columns of a quarter as 16-byte stores.
+// Swap-AB GEMM per (head h, 128-column chunk of c, tile of up to 128 rows b):
+//   D[c, b] = sum_d W_UK[h, d, c] * q_nope[b, h, d]
+// M = 128 (c), N = batch tile (multiple of 16), K = 128 (d).
+// A = W_UK[h][:, chunk] is M-major in memory (c contiguous): two TMA boxes of
+// 64 c x 128 d, 128B-swizzled.  B = q_nope[:, h, :] is K-major: two 3-D TMA
+// boxes of 64 d x N rows.  The accumulator lives in TMEM (lanes = c).
 // =============================================================================
-constexpr int kAbsorbRows = 128;
-constexpr int kAbsorbSmemA = 2 * kAbsorbRows * 128;                  // q_nope tile: 32 KB
-constexpr int kAbsorbSmemB = 4 * 64 * 128 * 2;                       // W_UK half: 64 KB
-constexpr int kAbsorbSmemBytes = kAbsorbSmemA + kAbsorbSmemB + 256 + kSmemAlignPad;  // + barriers
+constexpr int kAbsorbNMax = 128;
+constexpr int kAbsorbSmemA = 2 * 64 * 128 * 2;                      // 32 KB
+// shared memory for a batch tile of n rows: W_UK chunk, q_nope tile, barriers
+// (sized to the tile so that four CTAs fit on an SM when n <= 64)
+__host__ __device__ constexpr int absorb_smem_bytes(int n) { return kAbsorbSmemA + 2 * n * 128 + 256 + kSmemAlignPad; }
+constexpr int kAbsorbSmemBytes = absorb_smem_bytes(kAbsorbNMax);
 
 __global__ void __launch_bounds__(128, 1)
 absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
-              __nv_bfloat16* __restrict__ q_lat, int B, int* d_status) {
+              __nv_bfloat16* __restrict__ q_lat, int B, int n_tile, int* d_status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int half = blockIdx.x;  // latent columns [256 half, 256 half + 256)
+  const int chunk = blockIdx.x;  // 128-wide chunk of the latent dimension
   const int h = blockIdx.y;
-  const int b0 = blockIdx.z * kAbsorbRows;
+  const int b0 = blockIdx.z * kAbsorbNMax;
 
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + kAbsorbSmemA;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAbsorbSmemA + kAbsorbSmemB);
-  const uint32_t bar_load[2] = {smem_u32(&bars[0]), smem_u32(&bars[1])};
-  const uint32_t bar_mma[2] = {smem_u32(&bars[2]), smem_u32(&bars[3])};
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[4]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[5]);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAbsorbSmemA + 2 * n_tile * 128);
+  const uint32_t bar_load = smem_u32(&bars[0]);
+  const uint32_t bar_mma = smem_u32(&bars[1]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[3]);
   const AbortState ab{abort_flag, d_status};
 
+  const uint32_t tmem_cols = n_tile <= 32 ? 32u : (n_tile <= 64 ? 64u : 128u);
+  // The loads go out first (TMA needs no TMEM); TMEM is allocated meanwhile.
   if (tid == 0) {
     *abort_flag = 0;
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_load[i], 1);
-      mbar_init(bar_mma[i], 1);
-    }
+    mbar_init(bar_load, 1);
+    mbar_init(bar_mma, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_arrive_expect_tx(bar_load, kAbsorbSmemA + 2 * n_tile * 128);
+    const int wrow = h * kHeadRows;  // W_UK rows of head h
+    tma_load_2d(sA, &tm_w, bar_load, chunk * 128, wrow);
+    tma_load_2d(sA + 64 * 128 * 2, &tm_w, bar_load, chunk * 128 + 64, wrow);
+    tma_load_3d(sB, &tm_q, bar_load, 0, h, b0);
+    tma_load_3d(sB + n_tile * 128, &tm_q, bar_load, 64, h, b0);
+    grid_dep_launch();  // the attention kernel may start gathering
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_alloc(smem_u32(tmem_slot), tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -91,60 +96,40 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
   const uint32_t tmem = *tmem_slot;
 
   if (tid == 0) {
-    tma_prefetch_desc(&tm_w);
-    tma_prefetch_desc(&tm_q);
-    const int wrow = h * kHeadRows;  // W_UK rows of head h
-    // quarter 0: the query tile and the first two W boxes; quarter 1: the other two
-    mbar_arrive_expect_tx(bar_load[0], kAbsorbSmemA + 2 * 64 * 128 * 2);
-    tma_load_3d(sA, &tm_q, bar_load[0], 0, h, b0);
-    tma_load_3d(sA + kAbsorbRows * 128, &tm_q, bar_load[0], 64, h, b0);
-    mbar_arrive_expect_tx(bar_load[1], 2 * 64 * 128 * 2);
-    for (int box = 0; box < 4; ++box)
-      tma_load_2d(sB + box * (64 * 128 * 2), &tm_w, bar_load[box >> 1], half * 256 + box * 64, wrow);
-    grid_dep_launch();  // the attention kernel may start gathering
-
-    constexpr uint32_t idesc = idesc_bf16_f32(128, 128, /*a MN*/ false, /*b MN*/ true);
-    for (int qtr = 0; qtr < 2; ++qtr) {
-      wait(bar_load[qtr], 0, ab);
-      tc_fence_after();
-      for (int k = 0; k < kDn / 16; ++k) {
-        // A: 32 bytes of d per step inside the 128-byte rows; the second
-        // 64-wide d block follows the first.
-        const uint64_t a = smem_desc_sw128(sA + (k >> 2) * (kAbsorbRows * 128) + (k & 3) * 32, 16, 1024);
-        // B: 16 d-rows per step (two 8-row groups 1024 B apart); the two
-        // 64-wide c blocks of the quarter are 16 KB apart.
-        const uint64_t bd = smem_desc_sw128(sB + qtr * (2 * 64 * 128 * 2) + k * 16 * 128, 64 * 128 * 2, 1024);
-        mma_ss(tmem + qtr * 128, a, bd, idesc, k > 0 ? 1u : 0u);
-      }
-      mma_commit(bar_mma[qtr]);
+    wait(bar_load, 0, ab);
+    tc_fence_after();
+    const uint32_t idesc = idesc_bf16_f32(128, n_tile, /*a MN*/ true, /*b MN*/ false);
+    for (int k = 0; k < kDn / 16; ++k) {
+      // A: 16 d-rows per step (two 8-row groups 1024 B apart); the two
+      // 64-wide c blocks are 16 KB apart.
+      const uint64_t a = smem_desc_sw128(sA + k * 16 * 128, 64 * 128 * 2, 1024);
+      // B: 32 bytes of d per step inside the 128-byte row; the second
+      // 64-wide d block follows the first.
+      const uint64_t b = smem_desc_sw128(sB + (k >> 2) * n_tile * 128 + (k & 3) * 32, 16, 1024);
+      mma_ss(tmem, a, b, idesc, k > 0 ? 1u : 0u);
     }
+    mma_commit(bar_mma);
   }
   __syncwarp();
 
-  // Epilogue: lane (32*warp + lane) holds row b, 128 f32 columns per quarter.
-  const int b = b0 + warp * 32 + lane;
-  for (int qtr = 0; qtr < 2; ++qtr) {
-    wait(bar_mma[qtr], 0, ab);
-    tc_fence_after();
-#pragma unroll 1
-    for (int cc = 0; cc < 4; ++cc) {
-      uint32_t v[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + qtr * 128 + cc * 32, v);
-      tmem_wait_ld();
-      if (b < B) {
-        uint4* dst = reinterpret_cast<uint4*>(q_lat + ((size_t)b * kH + h) * kDl + half * 256 + qtr * 128 + cc * 32);
+  // Epilogue: lane (32*warp + lane) holds column c of the chunk, one TMEM
+  // column per batch row.
+  wait(bar_mma, 0, ab);
+  tc_fence_after();
+  const int c = chunk * 128 + warp * 32 + lane;
+  for (int n0 = 0; n0 < n_tile; n0 += 16) {
+    uint32_t v[16];
+    tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + n0, v);
+    tmem_wait_ld();
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
-          dst[t] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * t]), __uint_as_float(v[8 * t + 1])),
-                              pack_bf16x2(__uint_as_float(v[8 * t + 2]), __uint_as_float(v[8 * t + 3])),
-                              pack_bf16x2(__uint_as_float(v[8 * t + 4]), __uint_as_float(v[8 * t + 5])),
-                              pack_bf16x2(__uint_as_float(v[8 * t + 6]), __uint_as_float(v[8 * t + 7])));
-      }
+    for (int j = 0; j < 16; ++j) {
+      const int b = b0 + n0 + j;
+      if (b < B) q_lat[((size_t)b * kH + h) * kDl + c] = __float2bfloat16_rn(__uint_as_float(v[j]));
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 256);
+  if (warp == 0) tmem_dealloc(tmem, tmem_cols);
 }
 
 // =============================================================================

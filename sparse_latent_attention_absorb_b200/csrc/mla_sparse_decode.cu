@@ -194,13 +194,14 @@ int launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cuda
 }
 
 int launch_absorb(const void* q_nope, const void* wkv_b, void* q_lat, int B, int* d_status, cudaStream_t stream) {
+  const int n_tile = B >= kAbsorbNMax ? kAbsorbNMax : ceil_div(B, 16) * 16;
   CUtensorMap tm_w, tm_q;
   int rc;
   if ((rc = encode_wkv_b(&tm_w, wkv_b)) != MLA_OK) return rc;
-  if ((rc = encode_q_nope(&tm_q, q_nope, B, kAbsorbRows)) != MLA_OK) return rc;
-  dim3 grid(2, kH, ceil_div(B, kAbsorbRows));
-  return launch_ex(absorb_kernel, grid, dim3(128), kAbsorbSmemBytes, stream, false, tm_w, tm_q,
-                   static_cast<__nv_bfloat16*>(q_lat), B, d_status);
+  if ((rc = encode_q_nope(&tm_q, q_nope, B, n_tile)) != MLA_OK) return rc;
+  dim3 grid(kDl / 128, kH, ceil_div(B, kAbsorbNMax));
+  return launch_ex(absorb_kernel, grid, dim3(128), absorb_smem_bytes(n_tile), stream, false, tm_w, tm_q,
+                   static_cast<__nv_bfloat16*>(q_lat), B, n_tile, d_status);
 }
 
 int launch_attend(const void* q_lat, const void* q_pe, const void* kv_cache, const void* pe_cache,
