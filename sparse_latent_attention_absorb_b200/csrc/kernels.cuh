@@ -560,9 +560,14 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty));
-        float om = __uint_as_float(sv[0]);
+        // eight independent partial maxima (a 64-deep chain would be latency)
+        float om8[8];
 #pragma unroll
-        for (int t = 1; t < 64; ++t) om = fmaxf(om, __uint_as_float(sv[t]));
+        for (int u = 0; u < 8; ++u) om8[u] = __uint_as_float(sv[u]);
+#pragma unroll
+        for (int t = 8; t < 64; ++t) om8[t & 7] = fmaxf(om8[t & 7], __uint_as_float(sv[t]));
+        const float om = fmaxf(fmaxf(fmaxf(om8[0], om8[1]), fmaxf(om8[2], om8[3])),
+                               fmaxf(fmaxf(om8[4], om8[5]), fmaxf(om8[6], om8[7])));
         off = om * c2;  // c2 > 0: the maximum of the scaled values
 #pragma unroll
         for (int t = 0; t < 32; ++t)
@@ -602,7 +607,9 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       asm volatile("ld.shared.f32 %0, [%1];" : "=f"(off_peer) : "r"(x_mine + (uint32_t)(kXHalves + i * 4)) : "memory");
       const float base = off + off_peer;
       uint32_t sh[32];
-      __half2 hmx = __halves2half2(__ushort_as_half(0xfc00u), __ushort_as_half(0xfc00u));
+      __half2 hmx4[4];  // four independent partial maxima
+#pragma unroll
+      for (int e = 0; e < 4; ++e) hmx4[e] = __halves2half2(__ushort_as_half(0xfc00u), __ushort_as_half(0xfc00u));
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         uint32_t o[4];
@@ -616,11 +623,11 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
           memcpy(&a, &hv[4 * q + e], 4);
           memcpy(&p2, &o[e], 4);
           const __half2 sum = __hadd2(a, p2);
-          hmx = __hmax2(hmx, sum);
+          hmx4[e] = __hmax2(hmx4[e], sum);
           memcpy(&sh[4 * q + e], &sum, 4);
         }
       }
-      const float2 hm = __half22float2(hmx);
+      const float2 hm = __half22float2(__hmax2(__hmax2(hmx4[0], hmx4[1]), __hmax2(hmx4[2], hmx4[3])));
       const float mx = fmaxf(hm.x, hm.y) + base;  // the tile maximum (-inf if all masked)
       if (leader) MLA_TRACE_STAMP(kTrSmSummed, j);
       // Every lane has consumed its loads of the peer's push (the sums above
@@ -681,7 +688,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       // this group's P buffer was last read by PV(j-2)
       if (it > 0) wait(smem_u32(&bars->p_free[grp]), (it - 1) & 1, ab);
       tc_fence_after();
-      float lt = 0.f;
+      float lt4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent partial sums
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t pk[16];
@@ -691,11 +698,11 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
           const float p0 = ex2_approx(f.x - csub);
           const float p1 = ex2_approx(f.y - csub);
           pk[t] = pack_bf16x2(p0, p1);
-          lt += p0 + p1;
+          lt4[t & 3] += p0 + p1;
         }
         tmem_st16(pbuf + 16 * hh, pk);
       }
-      l_part += lt;
+      l_part += (lt4[0] + lt4[1]) + (lt4[2] + lt4[3]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
