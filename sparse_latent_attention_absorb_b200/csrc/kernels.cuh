@@ -292,7 +292,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
                      const __nv_bfloat16* __restrict__ kv_cache, const __nv_bfloat16* __restrict__ pe_cache,
                      const int32_t* __restrict__ end_pos, const int32_t* __restrict__ topk_idx, float scale,
                      void* __restrict__ o_part, float* __restrict__ lse_part, int K, int S_max, int n_split,
-                     int span, int* d_status) {
+                     int span, const __nv_bfloat16* __restrict__ w_next, int* d_status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -428,6 +428,16 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
         prefetch_tile(a0, a1);
         b0 = load_idx(j + 3 * kStages, 0);
         b1 = load_idx(j + 3 * kStages, 1);
+      }
+    }
+    // With its last tile gathered (a few tiles before this CTA ends), gather
+    // warp 0 pulls W_UV of head blockIdx.x (+ gridDim.x ...) into L2 for the
+    // value-up kernel that follows (w_next = wkv_b, or null to skip).
+    if (g == 0 && lane == 0 && w_next != nullptr) {
+      for (int hh = blockIdx.x; hh < kH; hh += gridDim.x) {
+        const __nv_bfloat16* w = w_next + (size_t)(hh * kHeadRows + kDn) * kDl;  // 128 rows x 512: 128 KB
+#pragma unroll
+        for (int part = 0; part < 4; ++part) prefetch_l2(w + part * 32 * kDl, 32 * kDl * 2);
       }
     }
   } else if (warp == kMmaWarp) {

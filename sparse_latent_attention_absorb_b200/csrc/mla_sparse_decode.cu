@@ -206,13 +206,15 @@ int launch_absorb(const void* q_nope, const void* wkv_b, void* q_lat, int B, int
 
 int launch_attend(const void* q_lat, const void* q_pe, const void* kv_cache, const void* pe_cache,
                   const int32_t* end_pos, const int32_t* topk_idx, float scale, void* o_part, float* lse_part, int B,
-                  int K, int S_max, int n_split, int span, int* d_status, cudaStream_t stream, bool pdl) {
+                  int K, int S_max, int n_split, int span, const void* w_next, int* d_status, cudaStream_t stream,
+                  bool pdl) {
   const long long ctas = 2LL * B * n_split;
   if (ctas > 0x7fffffffLL) return MLA_ERR_INVALID_ARG;
   return launch_ex(sparse_attend_kernel, dim3((unsigned)ctas), dim3(kAttendThreads), kAttendSmemBytes, stream, pdl,
                    static_cast<const __nv_bfloat16*>(q_lat), static_cast<const __nv_bfloat16*>(q_pe),
                    static_cast<const __nv_bfloat16*>(kv_cache), static_cast<const __nv_bfloat16*>(pe_cache), end_pos,
-                   topk_idx, scale, o_part, lse_part, K, S_max, n_split, span, d_status);
+                   topk_idx, scale, o_part, lse_part, K, S_max, n_split, span,
+                   static_cast<const __nv_bfloat16*>(w_next), d_status);
 }
 
 int launch_combine(const void* o_part, const float* lse_part, const void* wkv_b, void* out, float* lse_out, int B,
@@ -315,7 +317,7 @@ extern "C" int mla_sparse_attend(const void* q_lat, const void* q_pe, const void
   plan_splits(B, K, info->sm_count, &want, &span);
   if (n_split != want) return MLA_ERR_INVALID_ARG;
   return launch_attend(q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, scale, o_part, lse_part, B, K, S_max,
-                       n_split, span, d_status, stream, false);
+                       n_split, span, nullptr, d_status, stream, false);
 }
 
 extern "C" int mla_combine_value_up(const void* o_part, const float* lse_part, const void* wkv_b, void* out,
@@ -359,8 +361,10 @@ extern "C" int mla_sparse_decode(const void* q_nope, const void* q_pe, const voi
   // ordinary launch, so all earlier work in the stream (whatever wrote the
   // caches and indices) has finished before any of the three starts.
   if ((rc = launch_absorb(q_nope, wkv_b, q_lat, B, d_status, stream)) != MLA_OK) return rc;
+  // The attention kernel also pulls W_UV into L2 near its end, for the
+  // value-up kernel.
   if ((rc = launch_attend(q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, scale, o_part, lse_part, B, K, S_max,
-                          n_split, span, d_status, stream, true)) != MLA_OK)
+                          n_split, span, wkv_b, d_status, stream, true)) != MLA_OK)
     return rc;
   return launch_combine(o_part, lse_part, wkv_b, out, lse_out, B, n_split, d_status, stream, true);
 }
