@@ -80,7 +80,12 @@ int mla_num_splits(int B, int K);
 size_t mla_sparse_decode_workspace_size(int B, int K, int S_max);
 
 /*
- * The whole decode step (steps absorb .. value-up above).
+ * The whole decode step (steps absorb .. value-up above).  Three kernels on
+ * `stream`; the second and third are launched with a programmatic dependency
+ * on the one before them (each starts early and waits for its predecessor
+ * before reading that kernel's output), the first as an ordinary launch, so
+ * work enqueued on `stream` before the call has finished before any of them
+ * reads an input.
  *   q_nope   bf16 [B,128,128]   non-rotary queries
  *   q_pe     bf16 [B,128,64]    rotary queries, already rotated
  *   kv_cache bf16 [B,S_max,512] normalised latent cache c^KV

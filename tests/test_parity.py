@@ -292,6 +292,22 @@ def test_full_size_workloads_sampled_rows(name):
     torch.cuda.empty_cache()
 
 
+def test_more_rows_than_tiles_and_clusters():
+    """B = 150 rows of one split each: two row tiles in the absorption kernel,
+    more 2-CTA clusters than the GPU holds at once (a second wave), and three
+    row tiles in the value-up kernel, the last one ragged (22 rows, the rest
+    read as zero by TMA)."""
+    w = wl.Workload("t_b150_ctx200-300_top100", 150, 300, (200, 300), 100, "uniform", 3001)
+    d = wl.generate(w)
+    assert pkg.num_splits(150, 100) == 1
+    out, lse = gpu_decode(to_dev(d))
+    ref = run_oracle(d)
+    got = out.double().cpu().numpy()
+    assert np.all(np.isfinite(got))
+    assert np.max(np.abs(got - ref.out)) <= out_bound(ref.out)
+    assert np.max(np.abs(lse.double().cpu().numpy() - ref.lse)) <= 1e-2
+
+
 def test_online_softmax_rescales_when_scores_grow_along_the_tiles():
     """Scores that grow with position, visited in ascending order: the running
     maximum jumps by more than 2^8 on nearly every tile, so O is rescaled in
