@@ -359,42 +359,88 @@ def gpu_arm(args, rank, world, device):
     e2e = None
     if rank == 0 or world > 1:
         import sparse_latent_attention_absorb_b200 as api
-        hsets = []
-        for s in sets:
-            h = s["host"]
-            hsets.append({k: h[k].pin_memory() for k in ("q_nope", "q_pe", "end_pos", "topk_idx")})
-        dev_in = {k: torch.empty_like(sets[0][k]) for k in ("q_nope", "q_pe", "end_pos", "topk_idx")}
-        out_host = torch.empty((B, 128, 128), dtype=torch.bfloat16).pin_memory()
-        h2d = sum(v.numel() * v.element_size() for v in hsets[0].values())
-        d2h = out_host.numel() * out_host.element_size()
+        # Per step: the step's queries, end positions and indices cross from
+        # pinned host memory in one copy (packed), the decode runs through the
+        # public Python API, and the result is read back to pinned host
+        # memory.  Three streams pipeline consecutive steps: the upload of
+        # step i+1 and the read-back of step i-1 overlap the decode of step
+        # i (double-buffered device inputs and outputs, ordered by events).
+        names = ("q_nope", "q_pe", "end_pos", "topk_idx")
+        offs, off = {}, 0
+        for k in names:
+            offs[k] = off
+            off += -(-(sets[0][k].numel() * sets[0][k].element_size()) // 256) * 256
+        pack_bytes = off
+        hpack = []
+        for s_ in sets:
+            buf = torch.empty(pack_bytes, dtype=torch.uint8).pin_memory()
+            for k in names:
+                t = s_["host"][k].contiguous().view(torch.uint8).reshape(-1)
+                buf[offs[k]:offs[k] + t.numel()].copy_(t)
+            hpack.append(buf)
+        dpack = [torch.empty(pack_bytes, dtype=torch.uint8, device=device) for _ in range(2)]
+
+        def views(buf):
+            v = {}
+            for k in names:
+                ref = sets[0][k]
+                nbytes = ref.numel() * ref.element_size()
+                v[k] = buf[offs[k]:offs[k] + nbytes].view(ref.dtype).view(ref.shape)
+            return v
+
+        dviews = [views(b) for b in dpack]
+        douts = [torch.empty((B, 128, 128), dtype=torch.bfloat16, device=device) for _ in range(2)]
+        houts = [torch.empty((B, 128, 128), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        h2d = sum(sets[0][k].numel() * sets[0][k].element_size() for k in names)
+        d2h = houts[0].numel() * houts[0].element_size()
+        s_h2d, s_d2h = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
+        ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("h2d", "comp", "d2h")}
+        started = [False, False]
 
         def e2e_step(i):
-            for k, v in hsets[i].items():
-                dev_in[k].copy_(v, non_blocking=True)
-            api.mla_sparse_decode(dev_in["q_nope"], dev_in["q_pe"], sets[i]["kv_cache"], sets[i]["pe_cache"],
-                                  dev_in["end_pos"], dev_in["topk_idx"], sets[i]["wkv_b"], sets[i]["scale"],
-                                  out=outs[i], workspace=ws)
-            out_host.copy_(outs[i], non_blocking=True)
+            k, si = i % 2, i % NSETS
+            with torch.cuda.stream(s_h2d):
+                if started[k]:
+                    s_h2d.wait_event(ev["comp"][k])      # step i-2's decode has read this input slot
+                dpack[k].copy_(hpack[si], non_blocking=True)
+                ev["h2d"][k].record(s_h2d)
+            with torch.cuda.stream(stream):
+                stream.wait_event(ev["h2d"][k])
+                if started[k]:
+                    stream.wait_event(ev["d2h"][k])      # step i-2's result has been read back
+                v = dviews[k]
+                api.mla_sparse_decode(v["q_nope"], v["q_pe"], sets[si]["kv_cache"], sets[si]["pe_cache"],
+                                      v["end_pos"], v["topk_idx"], sets[si]["wkv_b"], sets[si]["scale"],
+                                      out=douts[k], workspace=ws, stream=stream)
+                ev["comp"][k].record(stream)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(ev["comp"][k])
+                houts[k].copy_(douts[k], non_blocking=True)
+                ev["d2h"][k].record(s_d2h)
+            started[k] = True
 
-        with torch.cuda.stream(stream):
-            for it in range(max(3, args.warmup)):
-                e2e_step(it % NSETS)
-        stream.synchronize()
+        for it in range(max(50, args.warmup)):  # host-side paths warm as well
+            e2e_step(it)
+        torch.cuda.synchronize()
         barrier()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            f0.record(stream)
-            for it in range(args.steps):
-                e2e_step(it % NSETS)
-            f1.record(stream)
-        stream.synchronize()
+        f0.record(s_h2d)
+        h0 = time.perf_counter()
+        for it in range(args.steps):
+            e2e_step(it)
+        host_ms = (time.perf_counter() - h0) * 1e3
+        f1.record(s_d2h)
+        torch.cuda.synchronize()
         e_ms = f0.elapsed_time(f1)
+        print(f"e2e: {args.steps} steps, host enqueue {host_ms:.1f} ms, device {e_ms:.1f} ms", file=sys.stderr)
         if world > 1:
             t = torch.tensor([e_ms], dtype=torch.float64, device=device)
             torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
             e_ms = float(t.item())
         e2e = {"value": B * world * args.steps / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h}
+               "d2h_bytes_per_step": d2h,
+               "how": "per step one packed pinned upload, mla_sparse_decode through the Python API, one read-back; "
+                      "three streams overlap consecutive steps"}
 
     # ---- roofline of the dominant kernel and of the whole call
     hbm, tf, tf_sus, kind = peaks()

@@ -64,15 +64,22 @@ def load_library():
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()
 
 
 def _stream(stream):
     s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+    return s.cuda_stream
 
 
 def _check(t: torch.Tensor, name: str, dtype, shape=None):
+    # one cheap test on the hot path; the detailed checks below only run to
+    # name what is wrong
+    try:
+        if t.is_cuda and t.dtype == dtype and (shape is None or t.shape == shape) and t.is_contiguous():
+            return
+    except AttributeError:
+        pass
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name}: expected a torch.Tensor")
     if not t.is_cuda:
@@ -90,12 +97,26 @@ def _raise(rc: int, where: str):
         raise MLAError(rc, where)
 
 
+_sizing_cache: dict = {}
+
+
 def num_splits(B: int, K: int) -> int:
-    return int(load_library().mla_num_splits(B, K))
+    """mla_num_splits for the current device (a pure function of the sizes and
+    the device's SM count, so it is cached)."""
+    key = ("splits", torch.cuda.current_device() if torch.cuda.is_available() else -1, B, K)
+    v = _sizing_cache.get(key)
+    if v is None:
+        v = _sizing_cache[key] = int(load_library().mla_num_splits(B, K))
+    return v
 
 
 def workspace_size(B: int, K: int, S_max: int) -> int:
-    return int(load_library().mla_sparse_decode_workspace_size(B, K, S_max))
+    """mla_sparse_decode_workspace_size for the current device (cached, as above)."""
+    key = ("ws", torch.cuda.current_device() if torch.cuda.is_available() else -1, B, K, S_max)
+    v = _sizing_cache.get(key)
+    if v is None:
+        v = _sizing_cache[key] = int(load_library().mla_sparse_decode_workspace_size(B, K, S_max))
+    return v
 
 
 def mla_sparse_decode(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, scale, out=None, workspace=None,
