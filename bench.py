@@ -359,77 +359,42 @@ def gpu_arm(args, rank, world, device):
     e2e = None
     if rank == 0 or world > 1:
         import sparse_latent_attention_absorb_b200 as api
-        # Per step: the step's queries, end positions and indices cross from
-        # pinned host memory in one copy (packed), the decode runs through the
-        # public Python API, and the result is read back to pinned host
-        # memory.  Three streams pipeline consecutive steps: the upload of
-        # step i+1 and the read-back of step i-1 overlap the decode of step
-        # i (double-buffered device inputs and outputs, ordered by events).
+        # Per step one call of the C ABI's host-buffer entry point (through
+        # the Python binding): the step's queries, end positions and indices
+        # are uploaded from pinned host memory, the decode runs, the result is
+        # read back to pinned host memory, all on the call's stream.  Steps
+        # alternate between two streams, each with its own workspace, so the
+        # copies of one step overlap the kernels of the next.
         names = ("q_nope", "q_pe", "end_pos", "topk_idx")
-        offs, off = {}, 0
-        for k in names:
-            offs[k] = off
-            off += -(-(sets[0][k].numel() * sets[0][k].element_size()) // 256) * 256
-        pack_bytes = off
-        hpack = []
-        for s_ in sets:
-            buf = torch.empty(pack_bytes, dtype=torch.uint8).pin_memory()
-            for k in names:
-                t = s_["host"][k].contiguous().view(torch.uint8).reshape(-1)
-                buf[offs[k]:offs[k] + t.numel()].copy_(t)
-            hpack.append(buf)
-        dpack = [torch.empty(pack_bytes, dtype=torch.uint8, device=device) for _ in range(2)]
-
-        def views(buf):
-            v = {}
-            for k in names:
-                ref = sets[0][k]
-                nbytes = ref.numel() * ref.element_size()
-                v[k] = buf[offs[k]:offs[k] + nbytes].view(ref.dtype).view(ref.shape)
-            return v
-
-        dviews = [views(b) for b in dpack]
-        douts = [torch.empty((B, 128, 128), dtype=torch.bfloat16, device=device) for _ in range(2)]
+        hins = [{k: s_["host"][k].contiguous().pin_memory() for k in names} for s_ in sets]
         houts = [torch.empty((B, 128, 128), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-        h2d = sum(sets[0][k].numel() * sets[0][k].element_size() for k in names)
+        hws = [torch.empty(api.host_workspace_size(B, K, S_max), dtype=torch.uint8, device=device) for _ in range(2)]
+        e2e_streams = [stream, torch.cuda.Stream(device=device)]
+        h2d = sum(hins[0][k].numel() * hins[0][k].element_size() for k in names)
         d2h = houts[0].numel() * houts[0].element_size()
-        s_h2d, s_d2h = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
-        ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("h2d", "comp", "d2h")}
-        started = [False, False]
 
         def e2e_step(i):
             k, si = i % 2, i % NSETS
-            with torch.cuda.stream(s_h2d):
-                if started[k]:
-                    s_h2d.wait_event(ev["comp"][k])      # step i-2's decode has read this input slot
-                dpack[k].copy_(hpack[si], non_blocking=True)
-                ev["h2d"][k].record(s_h2d)
-            with torch.cuda.stream(stream):
-                stream.wait_event(ev["h2d"][k])
-                if started[k]:
-                    stream.wait_event(ev["d2h"][k])      # step i-2's result has been read back
-                v = dviews[k]
-                api.mla_sparse_decode(v["q_nope"], v["q_pe"], sets[si]["kv_cache"], sets[si]["pe_cache"],
-                                      v["end_pos"], v["topk_idx"], sets[si]["wkv_b"], sets[si]["scale"],
-                                      out=douts[k], workspace=ws, stream=stream)
-                ev["comp"][k].record(stream)
-            with torch.cuda.stream(s_d2h):
-                s_d2h.wait_event(ev["comp"][k])
-                houts[k].copy_(douts[k], non_blocking=True)
-                ev["d2h"][k].record(s_d2h)
-            started[k] = True
+            h = hins[si]
+            api.mla_sparse_decode_host(h["q_nope"], h["q_pe"], h["end_pos"], h["topk_idx"], sets[si]["kv_cache"],
+                                       sets[si]["pe_cache"], sets[si]["wkv_b"], sets[si]["scale"], houts[k], hws[k],
+                                       stream=e2e_streams[k])
 
         for it in range(max(50, args.warmup)):  # host-side paths warm as well
             e2e_step(it)
         torch.cuda.synchronize()
         barrier()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(s_h2d)
+        side_done = torch.cuda.Event()
+        f0.record(e2e_streams[0])
+        e2e_streams[1].wait_event(f0)
         h0 = time.perf_counter()
         for it in range(args.steps):
             e2e_step(it)
         host_ms = (time.perf_counter() - h0) * 1e3
-        f1.record(s_d2h)
+        side_done.record(e2e_streams[1])
+        e2e_streams[0].wait_event(side_done)
+        f1.record(e2e_streams[0])
         torch.cuda.synchronize()
         e_ms = f0.elapsed_time(f1)
         print(f"e2e: {args.steps} steps, host enqueue {host_ms:.1f} ms, device {e_ms:.1f} ms", file=sys.stderr)
@@ -439,8 +404,8 @@ def gpu_arm(args, rank, world, device):
             e_ms = float(t.item())
         e2e = {"value": B * world * args.steps / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
-               "how": "per step one packed pinned upload, mla_sparse_decode through the Python API, one read-back; "
-                      "three streams overlap consecutive steps"}
+               "how": "per step one mla_sparse_decode_host call (pinned host inputs uploaded, decode, result read "
+                      "back on the call's stream); steps alternate between two streams"}
 
     # ---- roofline of the dominant kernel and of the whole call
     hbm, tf, tf_sus, kind = peaks()

@@ -180,6 +180,34 @@ int mla_sparse_decode_noalloc(const void* q_nope, const void* q_pe, const void* 
                               void* out, int B, int K, int S_max, float* lse_out, int* d_status,
                               cudaStream_t stream);
 
+/*
+ * The whole decode step with the per-call tensors in HOST memory: the
+ * queries, end positions and indices are read from, and the output written
+ * to, host buffers; the caches and wkv_b (model state) stay in device memory.
+ * The pages have no counterpart: this entry point exists for callers whose
+ * per-token inputs live on the host (a serving process that has not placed
+ * them on the device), so that one call covers upload, decode and read-back.
+ *   h_q_nope, h_q_pe, h_end_pos, h_topk_idx, h_out: host memory, layouts as in
+ *            mla_sparse_decode, 16-byte aligned; pinned (page-locked) memory
+ *            makes the copies asynchronous, other host memory also works but
+ *            the driver stages it
+ *   kv_cache, pe_cache, wkv_b, lse_out, d_status: device memory, as in
+ *            mla_sparse_decode
+ *   workspace / workspace_bytes: device scratch, 256-byte aligned, at least
+ *            mla_sparse_decode_host_workspace_size(B, K, S_max) bytes: the
+ *            decode's scratch plus device copies of the four inputs and out
+ * Enqueues on `stream`, in order: one cudaMemcpyAsync per input, the decode
+ * step, one cudaMemcpyAsync of out to h_out.  h_out is complete once `stream`
+ * has passed this point; the host buffers must stay valid until then.
+ * Consecutive calls overlap when they alternate between streams, each with
+ * its own workspace.  Returns an mla_status.
+ */
+size_t mla_sparse_decode_host_workspace_size(int B, int K, int S_max);
+int mla_sparse_decode_host(const void* h_q_nope, const void* h_q_pe, const int32_t* h_end_pos,
+                           const int32_t* h_topk_idx, const void* kv_cache, const void* pe_cache, const void* wkv_b,
+                           float scale, void* h_out, int B, int K, int S_max, void* workspace,
+                           size_t workspace_bytes, float* lse_out, int* d_status, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -22,7 +22,8 @@ STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_WORKSPACE", 3: "MLA
 
 # Every symbol the public header declares.
 EXPORTS = ("mla_status_string", "mla_num_splits", "mla_sparse_decode_workspace_size", "mla_sparse_decode",
-           "mla_absorb_q", "mla_sparse_attend", "mla_combine_value_up", "mla_sparse_decode_noalloc")
+           "mla_absorb_q", "mla_sparse_attend", "mla_combine_value_up", "mla_sparse_decode_noalloc",
+           "mla_sparse_decode_host_workspace_size", "mla_sparse_decode_host")
 STATIC_SCRATCH_BYTES = 32 << 20  # MLA_STATIC_SCRATCH_BYTES
 
 _lib = None
@@ -59,6 +60,10 @@ def load_library():
     lib.mla_combine_value_up.argtypes = [p, p, p, p, p, i, i, p]
     lib.mla_sparse_decode_noalloc.restype = i
     lib.mla_sparse_decode_noalloc.argtypes = [p, p, p, p, p, p, p, f, p, i, i, i, p, p, p]
+    lib.mla_sparse_decode_host_workspace_size.restype = sz
+    lib.mla_sparse_decode_host_workspace_size.argtypes = [i, i, i]
+    lib.mla_sparse_decode_host.restype = i
+    lib.mla_sparse_decode_host.argtypes = [p, p, p, p, p, p, p, f, p, i, i, i, p, sz, p, p, p]
     _lib = lib
     return lib
 
@@ -220,4 +225,45 @@ def mla_combine_value_up(o_part, lse_part, wkv_b, out=None, lse_out=None, stream
     rc = lib.mla_combine_value_up(_ptr(o_part), _ptr(lse_part), _ptr(wkv_b), _ptr(out), _ptr(lse_out), B, n_split,
                                   _stream(stream))
     _raise(rc, "mla_combine_value_up")
+    return out
+
+
+def host_workspace_size(B: int, K: int, S_max: int) -> int:
+    """mla_sparse_decode_host_workspace_size for the current device (cached)."""
+    key = ("hws", torch.cuda.current_device() if torch.cuda.is_available() else -1, B, K, S_max)
+    v = _sizing_cache.get(key)
+    if v is None:
+        v = _sizing_cache[key] = int(load_library().mla_sparse_decode_host_workspace_size(B, K, S_max))
+    return v
+
+
+def _check_host(t: torch.Tensor, name: str, dtype, shape):
+    if (not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != dtype or t.shape != shape
+            or not t.is_contiguous()):
+        raise ValueError(f"{name}: expected a contiguous host tensor {dtype} {tuple(shape)}")
+
+
+def mla_sparse_decode_host(q_nope, q_pe, end_pos, topk_idx, kv_cache, pe_cache, wkv_b, scale, out, workspace,
+                           lse_out=None, d_status=None, stream=None):
+    """The decode step with the per-call tensors in host memory (pin them for
+    asynchronous copies): q_nope, q_pe, end_pos, topk_idx and out are CPU
+    tensors; kv_cache, pe_cache, wkv_b and the workspace live on the device.
+    Enqueued on `stream`; `out` is complete once the stream has passed it."""
+    lib = load_library()
+    B, K, S_max = q_nope.shape[0], topk_idx.shape[1], kv_cache.shape[1]
+    bf = torch.bfloat16
+    _check_host(q_nope, "q_nope", bf, (B, H, D_NOPE))
+    _check_host(q_pe, "q_pe", bf, (B, H, D_ROPE))
+    _check_host(end_pos, "end_pos", torch.int32, (B,))
+    _check_host(topk_idx, "topk_idx", torch.int32, (B, K))
+    _check_host(out, "out", bf, (B, H, D_V))
+    _check(kv_cache, "kv_cache", bf, (B, S_max, D_LAT))
+    _check(pe_cache, "pe_cache", bf, (B, S_max, D_ROPE))
+    _check(wkv_b, "wkv_b", bf, (H * (D_NOPE + D_V), D_LAT))
+    _check(workspace, "workspace", torch.uint8)
+    rc = lib.mla_sparse_decode_host(q_nope.data_ptr(), q_pe.data_ptr(), end_pos.data_ptr(), topk_idx.data_ptr(),
+                                    kv_cache.data_ptr(), pe_cache.data_ptr(), wkv_b.data_ptr(), float(scale),
+                                    out.data_ptr(), B, K, S_max, workspace.data_ptr(), workspace.numel(),
+                                    _ptr(lse_out), _ptr(d_status), _stream(stream))
+    _raise(rc, "mla_sparse_decode_host")
     return out

@@ -412,3 +412,78 @@ extern "C" int mla_sparse_decode_noalloc(const void* q_nope, const void* q_pe, c
   return mla_sparse_decode(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, scale, out, B, K, S_max,
                            scratch, (size_t)MLA_STATIC_SCRATCH_BYTES, lse_out, d_status, stream);
 }
+
+// ---------------------------------------------------------------- host-buffer entry
+// The decode step with the per-call tensors in host memory (see the header):
+// the workspace holds the decode scratch, then device staging copies of the
+// four inputs and the output.
+namespace {
+struct HostStaging {
+  size_t decode = 0, q_nope = 0, q_pe = 0, end_pos = 0, topk_idx = 0, out = 0, total = 0;
+};
+
+HostStaging host_staging(int B, int K, int n_split) {
+  HostStaging h;
+  size_t off = workspace_layout(B, n_split).total;
+  h.decode = 0;
+  h.q_nope = off;
+  off = round_up(off + (size_t)B * kH * kDn * 2, 256);
+  h.q_pe = off;
+  off = round_up(off + (size_t)B * kH * kDr * 2, 256);
+  h.end_pos = off;
+  off = round_up(off + (size_t)B * 4, 256);
+  h.topk_idx = off;
+  off = round_up(off + (size_t)B * K * 4, 256);
+  h.out = off;
+  off = round_up(off + (size_t)B * kH * kDv * 2, 256);
+  h.total = off;
+  return h;
+}
+}  // namespace
+
+extern "C" size_t mla_sparse_decode_host_workspace_size(int B, int K, int S_max) {
+  if (!sizes_ok(B, K, S_max)) return 0;
+  int n_split = 0, span = 0;
+  plan_splits(B, K, planning_sm_count(), &n_split, &span);
+  return host_staging(B, K, n_split).total;
+}
+
+extern "C" int mla_sparse_decode_host(const void* h_q_nope, const void* h_q_pe, const int32_t* h_end_pos,
+                                      const int32_t* h_topk_idx, const void* kv_cache, const void* pe_cache,
+                                      const void* wkv_b, float scale, void* h_out, int B, int K, int S_max,
+                                      void* workspace, size_t workspace_bytes, float* lse_out, int* d_status,
+                                      cudaStream_t stream) {
+  const void* ptrs[] = {h_q_nope, h_q_pe, h_end_pos, h_topk_idx, kv_cache, pe_cache, wkv_b, h_out};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  if (lse_out && (reinterpret_cast<uintptr_t>(lse_out) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (!sizes_ok(B, K, S_max) || !std::isfinite(scale)) return MLA_ERR_INVALID_ARG;
+  DeviceInfo* info = nullptr;
+  int rc = prepare(&info);
+  if (rc != MLA_OK) return rc;
+  int n_split = 0, span = 0;
+  plan_splits(B, K, info->sm_count, &n_split, &span);
+  const HostStaging hs = host_staging(B, K, n_split);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < hs.total)
+    return MLA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* d_q_nope = ws + hs.q_nope;
+  void* d_q_pe = ws + hs.q_pe;
+  int32_t* d_end_pos = reinterpret_cast<int32_t*>(ws + hs.end_pos);
+  int32_t* d_topk_idx = reinterpret_cast<int32_t*>(ws + hs.topk_idx);
+  void* d_out = ws + hs.out;
+  // one plain asynchronous copy per tensor (pinned host memory makes them
+  // truly asynchronous; pageable memory works but stages through the driver)
+  if (cudaMemcpyAsync(d_q_nope, h_q_nope, (size_t)B * kH * kDn * 2, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(d_q_pe, h_q_pe, (size_t)B * kH * kDr * 2, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(d_end_pos, h_end_pos, (size_t)B * 4, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(d_topk_idx, h_topk_idx, (size_t)B * K * 4, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  rc = mla_sparse_decode(d_q_nope, d_q_pe, kv_cache, pe_cache, d_end_pos, d_topk_idx, wkv_b, scale, d_out, B, K,
+                         S_max, ws, hs.q_nope, lse_out, d_status, stream);
+  if (rc != MLA_OK) return rc;
+  if (cudaMemcpyAsync(h_out, d_out, (size_t)B * kH * kDv * 2, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  return MLA_OK;
+}
