@@ -191,7 +191,7 @@ constexpr int kSoftmaxWarps = 8;                   // two groups of four
 constexpr int kMmaWarp = 8;     // TMEM allocation, QK issue
 constexpr int kPvWarp = 9;      // PV issue
 constexpr int kGatherWarp0 = 10;
-constexpr int kGatherWarps = kStages;  // gather warp g always fills stage g
+constexpr int kGatherWarps = 4;  // gather warp g fills rows 16g..16g+15 of every tile
 // 14 warps: at most 128 registers a thread (the warps spread over the four
 // SM sub-partitions, 16K registers each, two of which hold four warps).
 constexpr int kAttendThreads = 32 * (kGatherWarp0 + kGatherWarps);  // 448
@@ -206,16 +206,18 @@ static_assert(kStageBytes % 1024 == 0 && kOffX % 1024 == 0 && kOffQpe % 1024 == 
               "swizzle atoms");
 static_assert(kAttendSmemBytes <= 232448, "shared memory");
 static_assert(kColS + kNt <= kColP && kColP + kNt <= kColQ && kColQ + 128 <= kColO, "TMEM map");
-// Each gather warp owns one stage (tiles g, g+kStages, ...), so every wait on
-// a stage's kv_empty barrier is exactly one phase after the warp's previous
-// wait on it; with fewer stages than warps a waiter could run two phases
-// ahead of the barrier, where a parity test cannot tell the phases apart.
-static_assert(kGatherWarps == kStages, "one stage per gather warp");
+// Every gather warp copies its rows of every tile, in tile order: its wait
+// on a stage's kv_empty before tile j is for PV(j - kStages), which cannot
+// complete before this warp's own arrival for tile j - kStages, so successive
+// waits on one barrier are exactly one phase apart (a parity test cannot tell
+// phases two apart).  For the same reason a warp never arrives twice on one
+// phase of kv_full.
+static_assert(kGatherWarps * 16 == kNt, "sixteen rows of a tile per gather warp");
 static_assert(kMmaWarp == kSoftmaxWarps && kPvWarp == kMmaWarp + 1 && kGatherWarp0 == kPvWarp + 1, "warp roles");
 
 struct AttendBars {
   uint64_t q_full;              // softmax warps (8 arrivals) after storing Q
-  uint64_t kv_full[kStages];    // the tile's gather warp (1 arrival) once its copies landed
+  uint64_t kv_full[kStages];    // every gather warp (4 arrivals) once its copies of the tile landed
   uint64_t kv_empty[kStages];   // MMA commit after PV of the tile
   uint64_t s_full[2];           // MMA commit after QK of a tile of group g: partial scores ready
   uint64_t s_empty;             // the tile's group (4 arrivals) after reading the partial scores
@@ -224,7 +226,7 @@ struct AttendBars {
   uint64_t x_full[2];           // 1 local arrival + kXBytes of the peer group's st.async
   uint64_t x_free[2];           // 4 arrivals of the peer's group g once it has read our push
   uint64_t m_ready[2][4];       // group g, lane quarter q (1 arrival): running maximum published
-  uint32_t vmask[kStages][2];   // valid positions of the tile in each stage (bit n of word n/32)
+  uint16_t vmask[kStages][4];   // valid positions of the tile in each stage (bit n%16 of part n/16)
   uint32_t tmem_addr;
   int abort_flag;
 };
@@ -270,6 +272,17 @@ enum TraceEvent {
   kTrSmSummed,         //   full scores and tile maximum formed
   kTrSmReleased,       //   peer told that its push has been read
   kTrSmMaxIn,          //   other group's running maximum received
+  kTrGatherWoke,       // gather warp: its stage's previous tile released (wait returned)
+  kTrSRead0,           // softmax warp of lane quarter q (kTrSRead0 + q): scores read, s_empty arrived
+  kTrSRead1,
+  kTrSRead2,
+  kTrSRead3,
+  kTrPFull0,           // softmax warp of lane quarter q (kTrPFull0 + q): P written, p_full arrived
+  kTrPFull1,
+  kTrPFull2,
+  kTrPFull3,
+  kTrQkKv,             // MMA thread: the tile's rows have landed (wait returned)
+  kTrQkWoke,           // MMA thread: score buffer free (wait returned)
   kTrEvents
 };
 constexpr int kTraceTiles = 512;
@@ -321,7 +334,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     bars->abort_flag = 0;
     mbar_init(smem_u32(&bars->q_full), kSoftmaxWarps);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(smem_u32(&bars->kv_full[i]), 1);
+      mbar_init(smem_u32(&bars->kv_full[i]), kGatherWarps);
       mbar_init(smem_u32(&bars->kv_empty[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -351,84 +364,86 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
 
   if (warp >= kGatherWarp0) {
     // ------------------------------------------------------------ gather
-    // Gather warp g owns stage g and tiles g, g+4, g+8, ...; lane l handles
-    // positions l and l+32 of a tile.  Latent: one position per instruction
-    // (32 lanes x 16 bytes = this CTA's 256 columns); rotary: eight positions
-    // per instruction (this CTA's 32 columns).  A tile is published
-    // (kv_full) as soon as its own copies have landed.
+    // All four gather warps fill every tile: warp g copies rows
+    // [16g, 16g + 16) of it (latent: one row per instruction, 32 lanes x 16
+    // bytes = this CTA's 256 columns; rotary: eight rows per instruction, this
+    // CTA's 32 columns), so a freed stage is refilled by four warps at once.
+    // A tile is published (kv_full, one arrival per warp) once every warp's
+    // copies have landed.  Each warp visits the stages in tile order, so its
+    // successive waits on one stage's kv_empty are exactly one phase apart.
     const int g = warp - kGatherWarp0;
+    const int row0 = 16 * g;
     const __nv_bfloat16* kv_row0 = kv_cache + (size_t)b * S_max * kDl + rank * 256;
     const __nv_bfloat16* pe_row0 = pe_cache + (size_t)b * S_max * kDr + rank * 32;
-    auto load_idx = [&](int t, int half) -> int {
+    // Index of row 16g + (lane % 16) of tile 2p + lane / 16 (a pair of tiles
+    // per register), or -1 for a padding or out-of-range slot.
+    auto load_pair = [&](int pr) -> int {
+      const int t = 2 * pr + (lane >> 4);
       int v = -1;
       if (t < n_tiles) {
-        const int k = k_begin + t * kNt + half * 32 + lane;
+        const int k = k_begin + t * kNt + row0 + (lane & 15);
         if (k < k_end) v = __ldg(idx_row + k);
       }
       return (v >= 0 && v < ep) ? v : -1;
     };
-    auto gather_tile = [&](int j, int idx0, int idx1) {
-      const int st = g;
+    // tile j = 2p + h of the pair register `idx` (its rows in lanes 16h..16h+15)
+    auto gather_tile = [&](int j, int idx, int h) {
+      const int st = j % kStages;
       if (j >= kStages) wait(smem_u32(&bars->kv_empty[st]), ((j / kStages) - 1) & 1, ab);
+      if (lane == 0) MLA_TRACE_STAMP(kTrGatherWoke, j);
       const uint32_t stage = sStage + st * kStageBytes;
-#pragma unroll 8
-      for (int n = 0; n < kNt; ++n) {
-        const int pos = __shfl_sync(0xffffffffu, n < 32 ? idx0 : idx1, n & 31);
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        const int pos = __shfl_sync(0xffffffffu, idx, 16 * h + n);
         const size_t p = pos >= 0 ? (size_t)pos : 0;
-        const uint32_t dst = stage + (lane >> 3) * kLatBlock + sw128_offset(n, lane & 7);
+        const uint32_t dst = stage + (lane >> 3) * kLatBlock + sw128_offset(row0 + n, lane & 7);
         cp_async_16(dst, kv_row0 + p * kDl + lane * 8, pos >= 0 ? 16u : 0u);
       }
 #pragma unroll
-      for (int q = 0; q < kNt / 8; ++q) {
+      for (int q = 0; q < 2; ++q) {
         const int n = q * 8 + (lane >> 2), c = lane & 3;
-        const int pos = __shfl_sync(0xffffffffu, q < 4 ? idx0 : idx1, n & 31);
+        const int pos = __shfl_sync(0xffffffffu, idx, 16 * h + n);
         const size_t p = pos >= 0 ? (size_t)pos : 0;
-        const uint32_t dst = stage + 4 * kLatBlock + sw64_offset(n, c);
+        const uint32_t dst = stage + 4 * kLatBlock + sw64_offset(row0 + n, c);
         cp_async_16(dst, pe_row0 + p * kDr + c * 8, pos >= 0 ? 16u : 0u);
       }
       cp_async_commit();
       if (lane == 0) MLA_TRACE_STAMP(kTrGatherIssue, j);
-      const uint32_t valid0 = __ballot_sync(0xffffffffu, idx0 >= 0);
-      const uint32_t valid1 = __ballot_sync(0xffffffffu, idx1 >= 0);
+      const uint32_t valid = (__ballot_sync(0xffffffffu, idx >= 0) >> (16 * h)) & 0xffffu;
       cp_async_wait_all();
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        bars->vmask[st][0] = valid0;  // published by the arrival below
-        bars->vmask[st][1] = valid1;
+        bars->vmask[st][g] = (uint16_t)valid;  // published by the arrival below
         mbar_arrive(smem_u32(&bars->kv_full[st]));
         MLA_TRACE_STAMP(kTrGatherLanded, j);
       }
     };
-    // Rows of this warp's next tile are pulled into L2 while the tile ahead
-    // of it is still in use, so its copies hit L2 once the stage frees.
-    auto prefetch_tile = [&](int idx0, int idx1) {
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        const int pos = h2 ? idx1 : idx0;
-        if (pos >= 0) {
-          const char* r = reinterpret_cast<const char*>(kv_row0 + (size_t)pos * kDl);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) asm volatile("prefetch.global.L2 [%0];" ::"l"(r + c * 128));
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(pe_row0 + (size_t)pos * kDr));
-        }
+    // This warp's rows of tile j are pulled into L2 four tiles ahead of their
+    // copies (lanes 16h..16h+15 of the pair register hold them).
+    auto prefetch_tile = [&](int idx, int h) {
+      const int pos = __shfl_sync(0xffffffffu, idx, 16 * h + (lane & 15));
+      if (pos >= 0) {
+        const char* r = reinterpret_cast<const char*>(kv_row0 + (size_t)pos * kDl) + (lane >> 4) * 256;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(r));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(r + 128));
+        if (lane < 16) asm volatile("prefetch.global.L2 [%0];" ::"l"(pe_row0 + (size_t)pos * kDr));
       }
     };
-    // this warp's next two tiles, statically indexed (a register copy of a
-    // pending load would wait for the load)
-    int a0 = load_idx(g, 0), a1 = load_idx(g, 1);
-    int b0 = load_idx(g + kStages, 0), b1 = load_idx(g + kStages, 1);
-    for (int j = g; j < n_tiles; j += 2 * kStages) {
-      gather_tile(j, a0, a1);
-      prefetch_tile(b0, b1);
-      a0 = load_idx(j + 2 * kStages, 0);
-      a1 = load_idx(j + 2 * kStages, 1);
-      if (j + kStages < n_tiles) {
-        gather_tile(j + kStages, b0, b1);
-        prefetch_tile(a0, a1);
-        b0 = load_idx(j + 3 * kStages, 0);
-        b1 = load_idx(j + 3 * kStages, 1);
+    // index registers: tiles (2p, 2p+1), (2p+2, 2p+3), (2p+4, 2p+5); each is
+    // loaded a pair ahead of its first use (a register copy of a pending load
+    // would wait for the load)
+    int cur = load_pair(0), nxt = load_pair(1), pf = load_pair(2);
+    for (int pr = 0; 2 * pr < n_tiles; ++pr) {
+      gather_tile(2 * pr, cur, 0);
+      prefetch_tile(pf, 0);
+      if (2 * pr + 1 < n_tiles) {
+        gather_tile(2 * pr + 1, cur, 1);
+        prefetch_tile(pf, 1);
       }
+      cur = nxt;
+      nxt = pf;
+      pf = load_pair(pr + 3);
     }
     // With its last tile gathered (a few tiles before this CTA ends), gather
     // warp 0 pulls W_UV of head blockIdx.x (+ gridDim.x ...) into L2 for the
@@ -454,7 +469,9 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       wait(smem_u32(&bars->q_full), 0, ab);
       for (int qk = 0, st = 0; qk < n_tiles; ++qk, st = (st + 1 == kStages) ? 0 : st + 1) {
         wait(smem_u32(&bars->kv_full[st]), (qk / kStages) & 1, ab);
+        MLA_TRACE_STAMP(kTrQkKv, qk);
         if (qk > 0) wait(smem_u32(&bars->s_empty), (qk - 1) & 1, ab);
+        MLA_TRACE_STAMP(kTrQkWoke, qk);
         tc_fence_after();
         MLA_TRACE_STAMP(kTrQkStart, qk);
         const uint64_t dl = d_lat + (uint64_t)((st * kStageBytes) >> 4);
@@ -554,8 +571,9 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       // valid positions of tile j (the stage cannot be refilled before PV(j))
       const int st = j % kStages;
       wait(smem_u32(&bars->kv_full[st]), (j / kStages) & 1, ab);
+      // parts 0,1 and 2,3 read as two words: bit n of word n/32
       const uint32_t vm0 = *reinterpret_cast<volatile uint32_t*>(&bars->vmask[st][0]);
-      const uint32_t vm1 = *reinterpret_cast<volatile uint32_t*>(&bars->vmask[st][1]);
+      const uint32_t vm1 = *reinterpret_cast<volatile uint32_t*>(&bars->vmask[st][2]);
       // Our half in log2 units, as fp16 relative to its own maximum over the
       // tile (sent exactly, in fp32, beside it): the rounding then scales with
       // the spread of the scores inside the tile, not with their size.
@@ -569,7 +587,10 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty));
+        if (lane == 0) {
+          mbar_arrive(smem_u32(&bars->s_empty));
+          MLA_TRACE_STAMP(kTrSRead0 + qd, j);
+        }
         // eight independent partial maxima (a 64-deep chain would be latency)
         float om8[8];
 #pragma unroll
@@ -716,7 +737,10 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[grp]));
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&bars->p_full[grp]));
+        MLA_TRACE_STAMP(kTrPFull0 + qd, j);
+      }
       if (leader) MLA_TRACE_STAMP(kTrPWritten, j);
     }
 
