@@ -192,6 +192,13 @@ constexpr int kMmaWarp = 8;     // TMEM allocation, QK issue
 constexpr int kPvWarp = 9;      // PV issue
 constexpr int kGatherWarp0 = 10;
 constexpr int kGatherWarps = 4;  // gather warp g fills rows 16g..16g+15 of every tile
+// PV(j) is issued after QK(j + kPvLag).  QK(j + kPvLag) needs the stage of
+// tile j + kPvLag - kStages, freed by that tile's PV: it must come before
+// PV(j), or PV(j) would wait for itself.  A lag of 3 keeps PV out of the QK
+// it used to interleave with, but then the stage of tile j + 1 frees only
+// after QK(j): the ring, not the score buffer, sets the pace.
+constexpr int kPvLag = 2;
+static_assert(kPvLag < kStages, "PV may not wait for a QK that needs its own stage");
 // 14 warps: at most 128 registers a thread (the warps spread over the four
 // SM sub-partitions, 16K registers each, two of which hold four warps).
 constexpr int kAttendThreads = 32 * (kGatherWarp0 + kGatherWarps);  // 448
@@ -229,6 +236,7 @@ struct AttendBars {
   uint16_t vmask[kStages][4];   // valid positions of the tile in each stage (bit n%16 of part n/16)
   uint32_t tmem_addr;
   int abort_flag;
+  int qk_issued;                // QK steps issued so far (written by the MMA thread)
 };
 static_assert(sizeof(AttendBars) <= kBarBytes, "barrier block");
 
@@ -332,6 +340,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
 
   if (tid == 0) {
     bars->abort_flag = 0;
+    bars->qk_issued = 0;
     mbar_init(smem_u32(&bars->q_full), kSoftmaxWarps);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&bars->kv_full[i]), kGatherWarps);
@@ -485,6 +494,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
         for (int k = 0; k < 2; ++k)  // rotary: 32 bytes per step inside the 64-byte rows
           mma_ss(dst, d_qpe + (uint64_t)((k * 32) >> 4), dr + (uint64_t)((k * 32) >> 4), idesc_qk, 1u);
         mma_commit(smem_u32(&bars->s_full[qk & 1]));
+        *reinterpret_cast<volatile int*>(&bars->qk_issued) = qk + 1;
         MLA_TRACE_STAMP(kTrQkIssued, qk);
       }
     }
@@ -498,6 +508,10 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       const uint64_t d_v = smem_desc_sw128(sStage, kLatBlock, 1024);  // PV B, latent, N-major
       for (int pv = 0, st = 0; pv < n_tiles; ++pv, st = (st + 1 == kStages) ? 0 : st + 1) {
         wait(smem_u32(&bars->p_full[pv & 1]), (pv >> 1) & 1, ab);
+        // The score buffer's loop (QK -> softmax reads S -> next QK) sets the
+        // pace, and the tensor pipe runs MMAs in issue order: PV(pv) enters
+        // it only once QK(pv + kPvLag) has been issued, behind that QK.
+        wait_counter(&bars->qk_issued, min(pv + kPvLag + 1, n_tiles), ab);
         tc_fence_after();
         MLA_TRACE_STAMP(kTrPvStart, pv);
         const uint64_t dv = d_v + (uint64_t)((st * kStageBytes) >> 4);

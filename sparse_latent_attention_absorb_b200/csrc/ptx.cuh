@@ -140,6 +140,28 @@ __device__ __forceinline__ bool wait_cluster(uint32_t bar, uint32_t parity, Abor
   return wait_slow(bar, parity, ab, true);
 }
 
+// Bounded wait until a shared-memory counter written by another thread of
+// this CTA reaches `target` (a scheduling condition: no data is handed over).
+__device__ __noinline__ bool wait_counter_slow(const volatile int* counter, int target, AbortState ab) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (*counter >= target) return true;
+    if ((it & 63u) == 63u) {
+      if (*ab.flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        *ab.flag = 1;
+        if (ab.status) atomicCAS(ab.status, 0, MLA_ERR_DEVICE_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ bool wait_counter(const volatile int* counter, int target, AbortState ab) {
+  if (*counter >= target) return true;
+  return wait_counter_slow(counter, target, ab);
+}
+
 // ----------------------------------------------------------------------------
 // cp.async (16-byte, L2 only) and proxy fences
 
