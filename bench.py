@@ -355,6 +355,21 @@ def gpu_arm(args, rank, world, device):
     t_attend = time_kernel(k_attend, reps)
     t_combine = time_kernel(k_combine, reps)
 
+    # ---- the step after the path: the output projection of the decode
+    # outputs (page "Attention update"), wo [7168, 16384] bf16 = 235 MB, more
+    # than L2, so every call streams it from HBM
+    p_dim = wl.D_MODEL
+    p_wo = wl.generate_projection(1, p_dim, seed=5001)["wo"].to(device)
+    p_delta = torch.empty((B, p_dim), dtype=torch.bfloat16, device=device)
+    p_ws = torch.empty(lib.mla_output_projection_workspace_size(B, p_dim), dtype=torch.uint8, device=device)
+
+    def k_project(i):
+        return lib.mla_output_projection(P(outs[i]), P(p_wo), P(p_delta), B, p_dim, P(p_ws), p_ws.numel(), None, sv)
+
+    t_project = time_kernel(k_project, min(50, reps))
+    p_bytes = p_dim * 16384 * 2 + B * 16384 * 2 + B * p_dim * 2
+    del p_wo
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if rank == 0 or world > 1:
@@ -437,6 +452,11 @@ def gpu_arm(args, rank, world, device):
                           "bound": "hbm" if t_hbm >= t_tc else "tensor",
                           "peaks": {"hbm_gbs": hbm, "bf16_tflops": tf, "source": kind}},
         "kernels_ms": {"absorb": t_absorb, "sparse_attend": t_attend, "combine_value_up": t_combine},
+        "projection": {"what": "output projection delta = x . wo^T of the decode outputs, wo bf16 [7168, 16384]",
+                       "ms_per_call": t_project, "launches_per_call": 1 if p_ws.numel() <= 256 else 2,
+                       "roofline": {"bound": "hbm", "achieved": p_bytes / (t_project * 1e-3) / 1e9, "peak": hbm,
+                                    "unit": "GB/s", "frac": p_bytes / (t_project * 1e-3) / 1e9 / hbm,
+                                    "alg_bytes_per_call": p_bytes, "peak_source": f"{kind} hbm_gbs"}},
         "gpu_launches": launches,
         "e2e": e2e,
         "clocks": clocks.summary(),

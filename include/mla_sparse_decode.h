@@ -208,6 +208,48 @@ int mla_sparse_decode_host(const void* h_q_nope, const void* h_q_pe, const int32
                            float scale, void* h_out, int B, int K, int S_max, void* workspace,
                            size_t workspace_bytes, float* lse_out, int* d_status, cudaStream_t stream);
 
+/*
+ * Output projection (model.py 607-608 as shown on the atlas page "Attention
+ * update": the head outputs of a row are flattened and projected back to the
+ * model width by wo, a RowParallelLinear from 128*128 inputs to dim outputs;
+ * the pages show no bias):
+ *   delta[b, n] = bf16( sum_{k < 16384} x[b, k] * wo[n, k] )   (fp32 accumulate)
+ *   x     bf16 [B, 16384]  the decode output [B,128,128] of mla_sparse_decode,
+ *                          row-major (k = 128 h + e)
+ *   wo    bf16 [dim, 16384] the torch Linear weight, k contiguous
+ *   delta bf16 [B, dim]    Delta_attn of the pages ([B, 1, 7168] at dim 7168)
+ *   dim   model width: a multiple of 128, 128 <= dim <= 65536 (7168 on the pages)
+ *   workspace / workspace_bytes  device scratch, 256-byte aligned, at least
+ *            mla_output_projection_workspace_size(B, dim) bytes (f32 partial
+ *            sums; the result does not depend on its contents)
+ *   d_status optional device int, as in mla_sparse_decode
+ * Sizes: 1 <= B <= 2^20; wo is read once per 256 batch rows.  The sum over k
+ * is split across SMs and added up in a fixed order, so results are
+ * reproducible.  Enqueues two kernels on `stream` (an ordinary launch, then a
+ * reduction with a programmatic dependency on it; with at least as many
+ * 128 x 256 output tiles as SMs, one kernel).  Returns an mla_status.
+ * mla_output_projection_workspace_size returns 0 only for invalid sizes.
+ */
+size_t mla_output_projection_workspace_size(int B, int dim);
+int mla_output_projection(const void* x, const void* wo, void* delta, int B, int dim, void* workspace,
+                          size_t workspace_bytes, int* d_status, cudaStream_t stream);
+
+/*
+ * The decode step followed by the output projection, in one call:
+ * delta = mla_output_projection(mla_sparse_decode(...)).  Arguments as in the
+ * two calls; the per-head outputs stay in the workspace, which must hold at
+ * least mla_sparse_decode_project_workspace_size(B, K, S_max, dim) bytes
+ * (256-byte aligned).  The projection kernel is launched with a programmatic
+ * dependency on the value-up kernel, so its first wo stages are requested
+ * while the decode finishes (wo must not be written by the decode's inputs'
+ * producers in the meantime: it is model state).  Returns an mla_status.
+ */
+size_t mla_sparse_decode_project_workspace_size(int B, int K, int S_max, int dim);
+int mla_sparse_decode_project(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                              const int32_t* end_pos, const int32_t* topk_idx, const void* wkv_b, float scale,
+                              const void* wo, void* delta, int B, int K, int S_max, int dim, void* workspace,
+                              size_t workspace_bytes, float* lse_out, int* d_status, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -231,6 +231,39 @@ int oracle_mla_sparse_decode_f64(
     return fail ? -1 : 0;
 }
 
+/*
+ * Output projection (model.py 607-608, atlas page "Attention update"): the
+ * head outputs of a row, flattened to n_in = H * Dv values, are projected to
+ * the model width by wo (a Linear layer, weight [dim, n_in], no bias on the
+ * pages):
+ *   delta[b, n] = sum_{k < n_in} x[b, k] * wo[n, k]
+ * in double precision from the exact input values.  x [B, n_in], wo
+ * [dim, n_in] row-major, given as bfloat16 bit patterns or as double
+ * (in_bf16).  Rows `rows[0..n_rows)` of x are computed; result r is row
+ * rows[r], written to delta[r * dim .. r * dim + dim).  Returns 0, or -1 for
+ * a row index out of range.
+ */
+int oracle_output_projection_f64(const void *x, const void *wo, int in_bf16, int B, int n_in, int dim,
+                                 const int32_t *rows, int n_rows, double *delta)
+{
+    for (int r = 0; r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= B)
+            return -1;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int n = 0; n < dim; ++n) {
+        for (int r = 0; r < n_rows; ++r) {
+            const size_t xrow = (size_t)rows[r] * n_in, wrow = (size_t)n * n_in;
+            double acc = 0.0;
+            for (int k = 0; k < n_in; ++k)
+                acc += load_elem(x, xrow + k, in_bf16) * load_elem(wo, wrow + k, in_bf16);
+            delta[(size_t)r * dim + n] = acc;
+        }
+    }
+    return 0;
+}
+
 /* Number of OpenMP threads the oracle's parallel loop will use. */
 int oracle_num_threads(void)
 {

@@ -55,6 +55,8 @@ def _load():
             p, i,                        # rows n_rows
             p, p, p, p, p,               # out lse q_lat o_lat w_full
         ]
+        lib.oracle_output_projection_f64.restype = ctypes.c_int
+        lib.oracle_output_projection_f64.argtypes = [p, p, i, i, i, i, p, i, p]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -168,3 +170,35 @@ def mla_sparse_decode(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx,
     if rc != 0:
         raise RuntimeError(f"oracle failed with code {rc}")
     return OracleResult(out=out, lse=lse, q_lat=ql, o_lat=ol, w_full=wf)
+
+
+def output_projection(x, wo, rows=None) -> np.ndarray:
+    """delta[r, n] = sum_k x[rows[r], k] * wo[n, k] in float64 (the attention
+    update of the atlas page "Attention update", model.py 607-608).
+
+    ``x`` [B, n_in] (or [B, H, Dv], flattened per row) and ``wo`` [dim, n_in]:
+    both bfloat16 (torch) / uint16 bit patterns (numpy), or both float64.
+    Returns [len(rows), dim] (all rows by default).
+    """
+    try:
+        import torch
+        is_bf16 = isinstance(x, torch.Tensor) and x.dtype == torch.bfloat16
+    except ImportError:  # pragma: no cover
+        is_bf16 = False
+    if not is_bf16 and isinstance(x, np.ndarray) and x.dtype == np.uint16:
+        is_bf16 = True
+    B = int(x.shape[0])
+    n_in = 1
+    for d in x.shape[1:]:
+        n_in *= int(d)
+    dim = int(wo.shape[0])
+    assert int(np.prod(wo.shape[1:])) == n_in, "wo must be [dim, n_in]"
+    xa = _dense(x, is_bf16).reshape(B, n_in)
+    wa = _dense(wo, is_bf16).reshape(dim, n_in)
+    rows_a = _ints(np.arange(B) if rows is None else rows).reshape(-1)
+    out = np.zeros((int(rows_a.shape[0]), dim), np.float64)
+    rc = _load().oracle_output_projection_f64(_ptr(xa), _ptr(wa), int(is_bf16), B, n_in, dim,
+                                              _ptr(rows_a), int(rows_a.shape[0]), _ptr(out))
+    if rc != 0:
+        raise RuntimeError(f"oracle failed with code {rc}")
+    return out

@@ -16,6 +16,7 @@ import torch
 from .build import LIB_PATH
 
 H, D_NOPE, D_ROPE, D_LAT, D_V = 128, 128, 64, 512, 128
+D_MODEL = 7168  # model width of the pages (wo: 128 * 128 -> 7168)
 
 STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_WORKSPACE", 3: "MLA_ERR_CUDA",
           4: "MLA_ERR_DEVICE_TIMEOUT", 5: "MLA_ERR_BAD_INDEX", 6: "MLA_ERR_UNSUPPORTED"}
@@ -23,7 +24,9 @@ STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_WORKSPACE", 3: "MLA
 # Every symbol the public header declares.
 EXPORTS = ("mla_status_string", "mla_num_splits", "mla_sparse_decode_workspace_size", "mla_sparse_decode",
            "mla_absorb_q", "mla_sparse_attend", "mla_combine_value_up", "mla_sparse_decode_noalloc",
-           "mla_sparse_decode_host_workspace_size", "mla_sparse_decode_host")
+           "mla_sparse_decode_host_workspace_size", "mla_sparse_decode_host",
+           "mla_output_projection_workspace_size", "mla_output_projection",
+           "mla_sparse_decode_project_workspace_size", "mla_sparse_decode_project")
 STATIC_SCRATCH_BYTES = 32 << 20  # MLA_STATIC_SCRATCH_BYTES
 
 _lib = None
@@ -64,6 +67,14 @@ def load_library():
     lib.mla_sparse_decode_host_workspace_size.argtypes = [i, i, i]
     lib.mla_sparse_decode_host.restype = i
     lib.mla_sparse_decode_host.argtypes = [p, p, p, p, p, p, p, f, p, i, i, i, p, sz, p, p, p]
+    lib.mla_output_projection_workspace_size.restype = sz
+    lib.mla_output_projection_workspace_size.argtypes = [i, i]
+    lib.mla_output_projection.restype = i
+    lib.mla_output_projection.argtypes = [p, p, p, i, i, p, sz, p, p]
+    lib.mla_sparse_decode_project_workspace_size.restype = sz
+    lib.mla_sparse_decode_project_workspace_size.argtypes = [i, i, i, i]
+    lib.mla_sparse_decode_project.restype = i
+    lib.mla_sparse_decode_project.argtypes = [p, p, p, p, p, p, p, f, p, p, i, i, i, i, p, sz, p, p, p]
     _lib = lib
     return lib
 
@@ -267,3 +278,86 @@ def mla_sparse_decode_host(q_nope, q_pe, end_pos, topk_idx, kv_cache, pe_cache, 
                                     _ptr(lse_out), _ptr(d_status), _stream(stream))
     _raise(rc, "mla_sparse_decode_host")
     return out
+
+
+def projection_workspace_size(B: int, dim: int) -> int:
+    """mla_output_projection_workspace_size for the current device (cached)."""
+    key = ("pws", torch.cuda.current_device() if torch.cuda.is_available() else -1, B, dim)
+    v = _sizing_cache.get(key)
+    if v is None:
+        v = _sizing_cache[key] = int(load_library().mla_output_projection_workspace_size(B, dim))
+    return v
+
+
+def mla_output_projection(x, wo, delta=None, workspace=None, d_status=None, stream=None):
+    """delta = x . wo^T (bf16 [B, dim]) for x bf16 [B,128,128] (or [B,16384])
+    and wo bf16 [dim, 16384]."""
+    lib = load_library()
+    B = x.shape[0]
+    dim = wo.shape[0]
+    bf = torch.bfloat16
+    if not (x.dim() == 2 and x.shape[1] == H * D_V):
+        _check(x, "x", bf, (B, H, D_V))
+    _check(x, "x", bf)
+    _check(wo, "wo", bf, (dim, H * D_V))
+    if delta is None:
+        delta = torch.empty((B, dim), dtype=bf, device=x.device)
+    _check(delta, "delta", bf, (B, dim))
+    if d_status is not None:
+        _check(d_status, "d_status", torch.int32, (1,))
+    if workspace is None:
+        need = projection_workspace_size(B, dim)
+        if need == 0:
+            raise MLAError(1, "mla_output_projection")
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check(workspace, "workspace", torch.uint8)
+    rc = lib.mla_output_projection(_ptr(x), _ptr(wo), _ptr(delta), B, dim, _ptr(workspace), workspace.numel(),
+                                   _ptr(d_status), _stream(stream))
+    _raise(rc, "mla_output_projection")
+    return delta
+
+
+def project_workspace_size(B: int, K: int, S_max: int, dim: int) -> int:
+    """mla_sparse_decode_project_workspace_size for the current device (cached)."""
+    key = ("dpws", torch.cuda.current_device() if torch.cuda.is_available() else -1, B, K, S_max, dim)
+    v = _sizing_cache.get(key)
+    if v is None:
+        v = _sizing_cache[key] = int(load_library().mla_sparse_decode_project_workspace_size(B, K, S_max, dim))
+    return v
+
+
+def mla_sparse_decode_project(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, scale, wo, delta=None,
+                              workspace=None, lse_out=None, d_status=None, stream=None):
+    """The decode step followed by the output projection; returns delta
+    (bf16 [B, dim], dim = wo.shape[0])."""
+    lib = load_library()
+    B, S_max, K = q_nope.shape[0], kv_cache.shape[1], topk_idx.shape[1]
+    dim = wo.shape[0]
+    bf = torch.bfloat16
+    _check(q_nope, "q_nope", bf, (B, H, D_NOPE))
+    _check(q_pe, "q_pe", bf, (B, H, D_ROPE))
+    _check(kv_cache, "kv_cache", bf, (B, S_max, D_LAT))
+    _check(pe_cache, "pe_cache", bf, (B, S_max, D_ROPE))
+    _check(end_pos, "end_pos", torch.int32, (B,))
+    _check(topk_idx, "topk_idx", torch.int32, (B, K))
+    _check(wkv_b, "wkv_b", bf, (H * (D_NOPE + D_V), D_LAT))
+    _check(wo, "wo", bf, (dim, H * D_V))
+    if delta is None:
+        delta = torch.empty((B, dim), dtype=bf, device=q_nope.device)
+    _check(delta, "delta", bf, (B, dim))
+    if lse_out is not None:
+        _check(lse_out, "lse_out", torch.float32, (B, H))
+    if d_status is not None:
+        _check(d_status, "d_status", torch.int32, (1,))
+    if workspace is None:
+        need = project_workspace_size(B, K, S_max, dim)
+        if need == 0:
+            raise MLAError(1, "mla_sparse_decode_project")
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_nope.device)
+    _check(workspace, "workspace", torch.uint8)
+    rc = lib.mla_sparse_decode_project(_ptr(q_nope), _ptr(q_pe), _ptr(kv_cache), _ptr(pe_cache), _ptr(end_pos),
+                                       _ptr(topk_idx), _ptr(wkv_b), float(scale), _ptr(wo), _ptr(delta), B, K,
+                                       S_max, dim, _ptr(workspace), workspace.numel(), _ptr(lse_out),
+                                       _ptr(d_status), _stream(stream))
+    _raise(rc, "mla_sparse_decode_project")
+    return delta

@@ -164,11 +164,11 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 //
 // Warp roles (448 threads): warps 0-3 softmax group 0 (even tiles), warps
 // 4-7 softmax group 1 (odd tiles), warp w covering TMEM lanes 32(w%4)..;
-// warp 8 TMEM allocation + QK issue; warp 9 PV issue; warps 10-13 gather (one
-// stage each).  QK and PV are issued by different threads: their MMAs
-// interleave in the tensor pipe, and a commit (which tracks the issuing
-// thread's MMAs only) signals PV completion without waiting for a QK queued
-// ahead of it.
+// warp 8 TMEM allocation + QK issue; warp 9 PV issue; warps 10-13 gather
+// (sixteen rows of every tile each).  QK and PV are issued by different
+// threads: their MMAs interleave in the tensor pipe, and a commit (which
+// tracks the issuing thread's MMAs only) signals PV completion without
+// waiting for a QK queued ahead of it.
 // =============================================================================
 constexpr int kNt = 64;                            // positions per tile
 constexpr int kStages = 4;                         // gathered tile ring
@@ -895,7 +895,8 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
       tma_load_2d(sA + kb * 128 * 128, &tm_w, bar_k(kb), kb * 64, wrow);
     }
   }
-  grid_dep_wait();  // o_part / lse_part come from the attention kernel
+  grid_dep_launch();  // a programmatically dependent successor (the output projection) may start
+  grid_dep_wait();    // o_part / lse_part come from the attention kernel
 
   if (n_split == 1) {
     // O~ rows b0.. of head h: eight boxes of 64 columns x n_tile rows (rows

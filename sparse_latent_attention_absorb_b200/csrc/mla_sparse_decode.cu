@@ -13,6 +13,7 @@
 
 #include "kernels.cuh"
 #include "mla_sparse_decode.h"
+#include "projection.cuh"
 
 namespace {
 
@@ -53,7 +54,8 @@ int current_device(DeviceInfo** info) {
     if (d.sm100) {
       if (cudaFuncSetAttribute(absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAbsorbSmemBytes) != cudaSuccess ||
           cudaFuncSetAttribute(sparse_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttendSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(combine_value_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCombineSmemBytes) != cudaSuccess)
+          cudaFuncSetAttribute(combine_value_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCombineSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(projection_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, proj_smem_max()) != cudaSuccess)
         return MLA_ERR_CUDA;
     }
     d.configured = true;
@@ -128,6 +130,32 @@ int encode_o_lat(CUtensorMap* m, const void* o_lat, int B, int n_tile) {
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// wo as a 2-D bf16 tensor [dim rows, 16384 columns], boxes of 64 columns x
+// 128 rows, 128-byte swizzle.
+int encode_wo(CUtensorMap* m, const void* wo, int dim) {
+  cuuint64_t dims[2] = {(cuuint64_t)kProjK, (cuuint64_t)dim};
+  cuuint64_t strides[1] = {(cuuint64_t)kProjK * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kProjKBlock, (cuuint32_t)kProjM};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(wo), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// The projection input x as a 2-D bf16 tensor [B rows, 16384 columns], boxes
+// of 64 columns x n_tile rows, 128-byte swizzle (rows past B read as zero).
+int encode_proj_x(CUtensorMap* m, const void* x, int B, int n_tile) {
+  cuuint64_t dims[2] = {(cuuint64_t)kProjK, (cuuint64_t)B};
+  cuuint64_t strides[1] = {(cuuint64_t)kProjK * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kProjKBlock, (cuuint32_t)n_tile};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- planning
 
 constexpr int kMaxB = 1 << 20;
@@ -148,6 +176,33 @@ void plan_splits(int B, int K, int sm_count, int* n_split, int* span) {
   const int sp = ceil_div(ceil_div(K, want), kNt) * kNt;
   *span = sp;
   *n_split = ceil_div(K, sp);
+}
+
+constexpr int kProjMaxDim = 1 << 16;
+
+bool proj_sizes_ok(int B, int dim) {
+  return B >= 1 && B <= kMaxB && dim >= kProjM && dim <= kProjMaxDim && dim % kProjM == 0;
+}
+
+// Output projection: batch tiles of at most 256 rows (equal, multiples of 16);
+// with fewer output tiles than SMs one CTA per SM shares the work unit by unit
+// (f32 partials, then the reduce kernel), otherwise one CTA per tile writes
+// bf16 directly.
+struct ProjPlan {
+  int n_tile = 0, tiles = 0, n_ctas = 0;
+  bool direct = false;
+  size_t partial_bytes = 0;
+};
+
+ProjPlan plan_projection(int B, int dim, int sm_count) {
+  ProjPlan p;
+  const int y_tiles = ceil_div(B, kProjNMax);
+  p.n_tile = ceil_div(ceil_div(B, y_tiles), 16) * 16;
+  p.tiles = y_tiles * (dim / kProjM);
+  p.direct = p.tiles >= sm_count;
+  p.n_ctas = p.direct ? p.tiles : sm_count;  // fewer CTAs than tiles x 256 units: a range spans <= 2 tiles
+  p.partial_bytes = p.direct ? 0 : (size_t)2 * p.n_ctas * p.n_tile * kProjM * sizeof(float);
+  return p;
 }
 
 struct WorkspaceLayout {
@@ -231,6 +286,26 @@ int launch_combine(const void* o_part, const float* lse_part, const void* wkv_b,
   dim3 grid(kH, ceil_div(B, kCombineNMax));
   return launch_ex(combine_value_up_kernel, grid, dim3(kCombineThreads), kCombineSmemBytes, stream, pdl, tm_w, tm_o,
                    o_part, lse_part, static_cast<__nv_bfloat16*>(out), lse_out, B, n_split, n_tile, d_status);
+}
+
+// projection_kernel, then (unless every CTA wrote its tile directly) the
+// reduce kernel with a programmatic dependency on it.  With pdl, the
+// projection kernel itself depends programmatically on the kernel before it:
+// it requests its first weight stages before waiting for that kernel.
+int launch_projection(const void* x, const void* wo, void* delta, int B, int dim, const ProjPlan& p, void* partial,
+                      int* d_status, cudaStream_t stream, bool pdl) {
+  CUtensorMap tm_wo, tm_x;
+  int rc;
+  if ((rc = encode_wo(&tm_wo, wo, dim)) != MLA_OK) return rc;
+  if ((rc = encode_proj_x(&tm_x, x, B, p.n_tile)) != MLA_OK) return rc;
+  if ((rc = launch_ex(projection_kernel, dim3((unsigned)p.n_ctas), dim3(kProjThreads), proj_smem_bytes(p.n_tile),
+                      stream, pdl, tm_wo, tm_x, static_cast<float*>(partial), static_cast<__nv_bfloat16*>(delta), B,
+                      dim, p.n_tile, p.n_ctas, p.direct ? 1 : 0, d_status)) != MLA_OK)
+    return rc;
+  if (p.direct) return MLA_OK;
+  dim3 grid((unsigned)p.tiles, ceil_div(p.n_tile, kProjReduceRows));
+  return launch_ex(projection_reduce_kernel, grid, dim3(kProjM), 0, stream, true, static_cast<const float*>(partial),
+                   static_cast<__nv_bfloat16*>(delta), B, dim, p.n_tile, p.n_ctas);
 }
 
 int prepare(DeviceInfo** info) {
@@ -486,4 +561,85 @@ extern "C" int mla_sparse_decode_host(const void* h_q_nope, const void* h_q_pe, 
   if (cudaMemcpyAsync(h_out, d_out, (size_t)B * kH * kDv * 2, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;
+}
+
+// ---------------------------------------------------------------- output projection
+// delta = x . wo^T (see the header).
+
+extern "C" size_t mla_output_projection_workspace_size(int B, int dim) {
+  if (!proj_sizes_ok(B, dim)) return 0;
+  const ProjPlan p = plan_projection(B, dim, planning_sm_count());
+  return p.partial_bytes > 0 ? p.partial_bytes : 256;  // never 0 for valid sizes
+}
+
+extern "C" int mla_output_projection(const void* x, const void* wo, void* delta, int B, int dim, void* workspace,
+                                     size_t workspace_bytes, int* d_status, cudaStream_t stream) {
+  const void* ptrs[] = {x, wo, delta};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (!proj_sizes_ok(B, dim)) return MLA_ERR_INVALID_ARG;
+  DeviceInfo* info = nullptr;
+  int rc = prepare(&info);
+  if (rc != MLA_OK) return rc;
+  const ProjPlan p = plan_projection(B, dim, info->sm_count);
+  const size_t need = p.partial_bytes > 0 ? p.partial_bytes : 256;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+    return MLA_ERR_WORKSPACE;
+  return launch_projection(x, wo, delta, B, dim, p, workspace, d_status, stream, false);
+}
+
+// The decode step followed by the output projection: the workspace holds the
+// decode scratch, the per-head outputs (bf16 [B,16384]) and the projection's
+// partials.
+namespace {
+struct ProjectLayout {
+  size_t decode = 0, out = 0, partial = 0, total = 0;
+};
+ProjectLayout project_layout(int B, int K, int dim, int sm_count) {
+  ProjectLayout l;
+  int n_split = 0, span = 0;
+  plan_splits(B, K, sm_count, &n_split, &span);
+  size_t off = round_up(workspace_layout(B, n_split).total, 256);
+  l.out = off;
+  off = round_up(off + (size_t)B * kProjK * 2, 256);
+  l.partial = off;
+  off = round_up(off + plan_projection(B, dim, sm_count).partial_bytes, 256);
+  l.total = off;
+  l.decode = l.out;
+  return l;
+}
+}  // namespace
+
+extern "C" size_t mla_sparse_decode_project_workspace_size(int B, int K, int S_max, int dim) {
+  if (!sizes_ok(B, K, S_max) || !proj_sizes_ok(B, dim)) return 0;
+  return project_layout(B, K, dim, planning_sm_count()).total;
+}
+
+extern "C" int mla_sparse_decode_project(const void* q_nope, const void* q_pe, const void* kv_cache,
+                                         const void* pe_cache, const int32_t* end_pos, const int32_t* topk_idx,
+                                         const void* wkv_b, float scale, const void* wo, void* delta, int B, int K,
+                                         int S_max, int dim, void* workspace, size_t workspace_bytes,
+                                         float* lse_out, int* d_status, cudaStream_t stream) {
+  const void* ptrs[] = {q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, wo, delta};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  if (lse_out && (reinterpret_cast<uintptr_t>(lse_out) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (!sizes_ok(B, K, S_max) || !proj_sizes_ok(B, dim) || !std::isfinite(scale)) return MLA_ERR_INVALID_ARG;
+  DeviceInfo* info = nullptr;
+  int rc = prepare(&info);
+  if (rc != MLA_OK) return rc;
+  const ProjectLayout l = project_layout(B, K, dim, info->sm_count);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < l.total)
+    return MLA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* out = ws + l.out;
+  rc = mla_sparse_decode(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, scale, out, B, K, S_max, ws,
+                         l.decode, lse_out, d_status, stream);
+  if (rc != MLA_OK) return rc;
+  // programmatic dependency on the value-up kernel: the first weight stages
+  // of wo stream in while it finishes
+  return launch_projection(out, wo, delta, B, dim, plan_projection(B, dim, info->sm_count), ws + l.partial,
+                           d_status, stream, true);
 }

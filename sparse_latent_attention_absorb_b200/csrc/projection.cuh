@@ -1,0 +1,261 @@
+// sm_100a kernels of the attention output projection (DeepSeek-V3.2-Exp,
+// model.py 607-608 as shown on the atlas page "Attention update"): the head
+// outputs of a row are flattened (128 heads x 128 value dimensions = 16384)
+// and projected back to the model width by wo:
+//
+//   delta[b, n] = bf16( sum_k x[b, k] * wo[n, k] ),   k < 16384, n < dim
+//
+// wo is the torch Linear weight [dim, 16384] (k contiguous); the pages show no
+// bias.  At decode sizes the projection is a stream over wo (235 MB at
+// dim = 7168) with a narrow batch, so it is written as a weight stream:
+//
+//   projection_kernel  persistent swap-AB tcgen05 GEMM.  An output tile is
+//                      (batch tile y of n_tile <= 256 rows, wo tile m of 128
+//                      rows); a work unit is (tile, k-block of 64): A = wo
+//                      box [128 x 64], B = x box [n_tile x 64], both by TMA
+//                      (128B swizzle) into a ring of stages; D[n, b] in TMEM.
+//                      With fewer tiles than SMs, CTA c takes the contiguous
+//                      unit range [c U / C, (c+1) U / C) of all U = tiles x
+//                      256 units, so every SM streams the same number of
+//                      weight bytes; a range covers at most two tiles
+//                      (segments), and each segment's accumulator (two TMEM
+//                      buffers, so the MMAs run on while the previous one
+//                      drains) goes to an f32 partial slot.  With at least as
+//                      many tiles as SMs, CTA c computes tile c whole and
+//                      writes bf16 directly ("direct").
+//   projection_reduce_kernel  sums the partial slots of each tile in a fixed
+//                      order (deterministic) and rounds to bf16.
+//
+// Warp roles of projection_kernel (192 threads): warps 0-3 drain the
+// accumulator (TMEM lane quarter = warp), warp 4 lane 0 issues TMA, warp 5
+// allocates TMEM and its lane 0 issues the MMAs.
+#pragma once
+
+#include "kernels.cuh"
+
+namespace mla {
+
+constexpr int kProjK = kH * kDv;                   // 16384 inputs per row
+constexpr int kProjKBlock = 64;                    // k per unit: one 128-byte swizzle row
+constexpr int kProjKBlocks = kProjK / kProjKBlock; // 256 units per row tile
+constexpr int kProjM = 128;                        // wo rows per tile (MMA M)
+constexpr int kProjNMax = 256;                     // batch rows per tile (MMA N, TMA box)
+constexpr int kProjStagesMax = 8;
+constexpr int kProjStageBudget = 200 * 1024;       // shared memory for the ring
+constexpr int kProjABytes = kProjM * kProjKBlock * 2;  // 16 KB
+constexpr int kProjThreads = 192;
+constexpr int kProjReduceRows = 16;                // batch rows per reduce CTA
+
+__host__ __device__ constexpr int proj_stage_bytes(int n_tile) { return kProjABytes + n_tile * kProjKBlock * 2; }
+__host__ __device__ constexpr int proj_stages(int n_tile) {
+  return kProjStageBudget / proj_stage_bytes(n_tile) < kProjStagesMax ? kProjStageBudget / proj_stage_bytes(n_tile)
+                                                                      : kProjStagesMax;
+}
+// shared memory of one CTA: the ring, barriers, alignment pad
+__host__ __device__ constexpr int proj_smem_bytes(int n_tile) {
+  return proj_stages(n_tile) * proj_stage_bytes(n_tile) + 256 + kSmemAlignPad;
+}
+// the largest of them, over the batch tiles the host can choose
+constexpr int proj_smem_max() {
+  int m = 0;
+  for (int n = 16; n <= kProjNMax; n += 16) m = proj_smem_bytes(n) > m ? proj_smem_bytes(n) : m;
+  return m;
+}
+static_assert(proj_smem_max() <= 232448, "shared memory");
+static_assert(proj_stages(kProjNMax) >= 2, "ring depth");
+
+// First unit of CTA c when U units are spread over C CTAs.
+__host__ __device__ __forceinline__ long long proj_unit_begin(long long c, long long U, long long C) {
+  return c * U / C;
+}
+// The CTA whose unit range contains unit x: the largest c with
+// proj_unit_begin(c) <= x, i.e. ceil((x + 1) C / U) - 1.
+__host__ __device__ __forceinline__ int proj_cta_of_unit(long long x, long long U, long long C) {
+  return (int)(((x + 1) * C - 1) / U);
+}
+
+__global__ void __launch_bounds__(kProjThreads, 1)
+projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_x,
+                  float* __restrict__ partial, __nv_bfloat16* __restrict__ delta, int B, int dim, int n_tile,
+                  int n_ctas, int direct, int* d_status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = align_smem_1024(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x;
+  const int stages = proj_stages(n_tile);
+  const int stage_bytes = proj_stage_bytes(n_tile);
+  const int m_tiles = dim / kProjM;
+  const long long U = (long long)m_tiles * ((B + n_tile - 1) / n_tile) * kProjKBlocks;
+  const long long u0 = proj_unit_begin(c, U, n_ctas);
+  const int n_units = (int)(proj_unit_begin(c + 1, U, n_ctas) - u0);
+  const long long t0 = u0 / kProjKBlocks;  // first tile of this CTA
+  const int n_seg = n_units > 0 ? (int)((u0 + n_units - 1) / kProjKBlocks - t0) + 1 : 0;  // <= 2
+  // unit u: tile u / 256 = y * m_tiles + m, k-block u % 256
+  auto unit_m = [&](long long u) { return (int)((u / kProjKBlocks) % m_tiles); };
+  auto unit_row0 = [&](long long u) { return (int)((u / kProjKBlocks) / m_tiles) * n_tile; };
+
+  const uint32_t sRing = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
+  auto full = [&](int s) { return smem_u32(&bars[s]); };
+  auto empty = [&](int s) { return smem_u32(&bars[kProjStagesMax + s]); };
+  auto acc_full = [&](int a) { return smem_u32(&bars[2 * kProjStagesMax + a]); };
+  auto acc_empty = [&](int a) { return smem_u32(&bars[2 * kProjStagesMax + 2 + a]); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2 * kProjStagesMax + 4]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[2 * kProjStagesMax + 5]);
+  const AbortState ab{abort_flag, d_status};
+  // one accumulator buffer: n_tile f32 columns, rounded to a power of two
+  const uint32_t acc_cols = n_tile <= 32 ? 32u : (n_tile <= 64 ? 64u : (n_tile <= 128 ? 128u : 256u));
+
+  if (tid == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < kProjStagesMax; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(acc_full(a), 1);
+      mbar_init(acc_empty(a), 4);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), 2 * acc_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0 && n_units > 0) {
+      tma_prefetch_desc(&tm_wo);
+      tma_prefetch_desc(&tm_x);
+      // The first stages' weights go out before the wait on the kernel that
+      // writes x (programmatic dependent launch): wo does not depend on it.
+      const int pre = n_units < stages ? n_units : stages;
+      for (int i = 0; i < pre; ++i) {
+        const long long u = u0 + i;
+        mbar_arrive_expect_tx(full(i), stage_bytes);
+        tma_load_2d(sRing + i * stage_bytes, &tm_wo, full(i), (int)(u % kProjKBlocks) * kProjKBlock,
+                    unit_m(u) * kProjM);
+      }
+      grid_dep_wait();
+      for (int i = 0; i < pre; ++i) {
+        const long long u = u0 + i;
+        tma_load_2d(sRing + i * stage_bytes + kProjABytes, &tm_x, full(i), (int)(u % kProjKBlocks) * kProjKBlock,
+                    unit_row0(u));
+      }
+      for (int i = pre, st = pre % stages; i < n_units; ++i, st = (st + 1 == stages) ? 0 : st + 1) {
+        const long long u = u0 + i;
+        wait(empty(st), ((i / stages) - 1) & 1, ab);
+        const uint32_t dst = sRing + st * stage_bytes;
+        mbar_arrive_expect_tx(full(st), stage_bytes);
+        const int kx = (int)(u % kProjKBlocks) * kProjKBlock;
+        tma_load_2d(dst, &tm_wo, full(st), kx, unit_m(u) * kProjM);
+        tma_load_2d(dst + kProjABytes, &tm_x, full(st), kx, unit_row0(u));
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0 && n_units > 0) {
+      const uint32_t idesc = idesc_bf16_f32(kProjM, n_tile, false, false);
+      int seg = 0;
+      for (int i = 0, st = 0; i < n_units; ++i, st = (st + 1 == stages) ? 0 : st + 1) {
+        const long long u = u0 + i;
+        const bool first = (i == 0) || (u % kProjKBlocks == 0);
+        const bool last = (i == n_units - 1) || ((u + 1) % kProjKBlocks == 0);
+        const int acc = seg & 1;
+        if (first && seg >= 2) wait(acc_empty(acc), ((seg - 2) >> 1) & 1, ab);
+        wait(full(st), (i / stages) & 1, ab);
+        tc_fence_after();
+        const uint32_t a0 = sRing + st * stage_bytes;
+        const uint32_t b0 = a0 + kProjABytes;
+#pragma unroll
+        for (int k = 0; k < kProjKBlock / 16; ++k) {  // 32 bytes of k per step inside the 128-byte rows
+          const uint64_t a = smem_desc_sw128(a0 + k * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(b0 + k * 32, 16, 1024);
+          mma_ss(tmem + acc * acc_cols, a, bd, idesc, (first && k == 0) ? 0u : 1u);
+        }
+        mma_commit(empty(st));
+        if (last) {
+          mma_commit(acc_full(acc));
+          ++seg;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ drain
+    // Thread (warp w, lane l) holds wo row 32w + l of the tile: one TMEM
+    // column per batch row.  Partial slot 2c + seg is laid out [batch row of
+    // the tile][128 wo rows]; a direct tile goes to delta in bf16.
+    const int nl = warp * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    for (int seg = 0; seg < n_seg; ++seg) {
+      const int acc = seg & 1;
+      const long long u_seg = (t0 + seg) * kProjKBlocks;
+      const int row0 = unit_row0(u_seg);
+      wait(acc_full(acc), (seg >> 1) & 1, ab);
+      tc_fence_after();
+      float* dst = partial + ((size_t)(2 * c + seg) * n_tile) * kProjM + nl;
+      __nv_bfloat16* dd = delta + (size_t)row0 * dim + (size_t)unit_m(u_seg) * kProjM + nl;
+      for (int j0 = 0; j0 < n_tile; j0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + lane_base + acc * acc_cols + j0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          if (row0 + j0 + j >= B) continue;
+          if (direct)
+            dd[(size_t)(j0 + j) * dim] = __float2bfloat16_rn(__uint_as_float(v[j]));
+          else
+            dst[(size_t)(j0 + j) * kProjM] = __uint_as_float(v[j]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty(acc));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  // every CTA has issued its partial stores: the reduce kernel may launch
+  // (it waits for this grid's completion before reading them)
+  grid_dep_launch();
+  if (warp == 5) tmem_dealloc(tmem, 2 * acc_cols);
+}
+
+// delta[b, 128 m + n] = bf16( sum over the CTAs c whose units cover the tile
+// (y, m), in increasing c, of their partial for it ).  Grid (tiles, row groups
+// of kProjReduceRows within a tile); thread n = wo row within the tile.
+__global__ void __launch_bounds__(kProjM)
+projection_reduce_kernel(const float* __restrict__ partial, __nv_bfloat16* __restrict__ delta, int B, int dim,
+                         int n_tile, int n_ctas) {
+  const int t = blockIdx.x;
+  const int m_tiles = dim / kProjM;
+  const int m = t % m_tiles;
+  const int row0 = (t / m_tiles) * n_tile;
+  const int j0 = blockIdx.y * kProjReduceRows;  // first row of this CTA within the tile
+  const int n = threadIdx.x;
+  const long long U = (long long)m_tiles * ((B + n_tile - 1) / n_tile) * kProjKBlocks;
+  const long long first_unit = (long long)t * kProjKBlocks;
+  const int c_lo = proj_cta_of_unit(first_unit, U, n_ctas);
+  const int c_hi = proj_cta_of_unit(first_unit + kProjKBlocks - 1, U, n_ctas);
+  grid_dep_wait();  // the partials come from projection_kernel
+  for (int r = 0; r < kProjReduceRows; ++r) {
+    const int j = j0 + r;
+    if (j >= n_tile || row0 + j >= B) break;
+    float acc = 0.f;
+    for (int cc = c_lo; cc <= c_hi; ++cc) {
+      const int seg = (proj_unit_begin(cc, U, n_ctas) / kProjKBlocks == t) ? 0 : 1;
+      acc += __ldg(partial + ((size_t)(2 * cc + seg) * n_tile + j) * kProjM + n);
+    }
+    delta[(size_t)(row0 + j) * dim + (size_t)m * kProjM + n] = __float2bfloat16_rn(acc);
+  }
+}
+
+}  // namespace mla

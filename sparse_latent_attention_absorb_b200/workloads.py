@@ -10,7 +10,9 @@ q_nope 128 wide, q_pe 64 wide, a 512-wide cached latent, a 64-wide cached
 rotary key, and wkv_b viewed as [128 heads, 256, 512].
 
 Distributions: q_nope, q_pe, kv_cache and pe_cache are bf16 draws of N(0,1);
-wkv_b is bf16(N(0,1) * 512**-0.5); scale = fp32(192**-0.5).  Every index row
+wkv_b is bf16(N(0,1) * 512**-0.5); scale = fp32(192**-0.5).  For the output
+projection that follows the step (wo: 16384 -> 7168, page "Attention update"),
+its input x is a bf16 draw of N(0,1) and wo is bf16(N(0,1) * 16384**-0.5).  Every index row
 holds distinct positions in [0, end_pos), shuffled (the indexer's top-k output
 is in score order, not position order), padded with -1 up to K.
 """
@@ -25,6 +27,7 @@ D_NOPE = 128     # qk_nope_head_dim
 D_ROPE = 64      # qk_rope_head_dim
 D_LAT = 512      # kv_lora_rank
 D_V = 128        # v_head_dim
+D_MODEL = 7168   # model width: wo maps H * D_V = 16384 -> 7168
 SCALE = float(torch.tensor((D_NOPE + D_ROPE) ** -0.5, dtype=torch.float32))
 
 
@@ -186,3 +189,14 @@ def selected_count(end_pos: torch.Tensor, topk_idx: torch.Tensor) -> int:
     ep = end_pos.to(torch.int64).unsqueeze(1)
     t = topk_idx.to(torch.int64)
     return int(((t >= 0) & (t < ep)).sum())
+
+
+def generate_projection(B: int, dim: int = D_MODEL, seed: int = 2001) -> dict:
+    """Inputs of one output projection, on the CPU: x bf16 [B, 16384] (the
+    flattened per-head outputs of B rows) and wo bf16 [dim, 16384]."""
+    gen = torch.Generator().manual_seed(seed)
+    n_in = H * D_V
+    return {
+        "x": _bf16_normal((B, n_in), gen),
+        "wo": _bf16_normal((dim, n_in), gen, std=n_in ** -0.5, chunk_dim0=dim * n_in > (1 << 26)),
+    }

@@ -13,7 +13,11 @@ a disagreement:
   output replaced by the given index row and the -inf/scatter mask built
   literally over all end_pos positions.
 
-Neither shares code with the oracle.
+* ``transcript_projection``: the output projection of the page "Attention
+  update" (model.py 607-608), ``self.wo(x.flatten(2))``, as torch's
+  ``F.linear`` in float64 on the [B, 1, H, Dv] head outputs.
+
+None shares code with the oracle.
 """
 from __future__ import annotations
 
@@ -85,3 +89,14 @@ def transcript(q_nope, q_pe, kv, pe, wkv_b, end_pos, topk_idx, scale, Dv=None):
         x = torch.einsum("bshc,hdc->bshd", x, wkv[:, -Dv:])
         outs.append(x[0, 0])
     return torch.stack(outs).numpy()
+
+
+def transcript_projection(x, wo):
+    """``wo(x.flatten(2))`` of the page "Attention update": x holds the head
+    outputs [B, H, Dv] of one position per row (or [B, H*Dv]); wo is the
+    Linear weight [dim, H*Dv].  Returns [B, dim] in float64."""
+    xt = torch.as_tensor(to_f64(x))
+    B = xt.shape[0]
+    x4 = xt.reshape(B, 1, -1, xt.shape[-1]) if xt.dim() == 3 else xt.reshape(B, 1, 1, -1)
+    w = torch.as_tensor(to_f64(wo))
+    return torch.nn.functional.linear(x4.flatten(2), w)[:, 0].numpy()

@@ -116,3 +116,65 @@ def test_binding_rejects_cpu_tensors():
     x = torch.zeros((1, 128, 128), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         binding.mla_absorb_q(x, torch.zeros((128 * 256, 512), dtype=torch.bfloat16))
+
+
+def test_projection_workspace_size_formula(lib):
+    sms = 148  # planning SM count without a visible GPU (B200)
+    for B, dim in ((1, 7168), (64, 7168), (3, 128), (256, 1024), (300, 256)):
+        y_tiles = -(-B // 256)
+        n_tile = -(-(-(-B // y_tiles)) // 16) * 16
+        tiles = y_tiles * (dim // 128)
+        got = lib.mla_output_projection_workspace_size(B, dim)
+        if tiles >= sms:
+            assert got == 256  # one CTA per tile writes bf16 directly: no partials
+        else:
+            assert got == 2 * sms * n_tile * 128 * 4  # two f32 partial slots per CTA
+    assert lib.mla_output_projection_workspace_size(1000, 7168) == 256  # 4 x 56 tiles >= 148 SMs
+    for B, dim in ((0, 7168), (1, 0), (1, 100), (1, 7169), (1, 1 << 17)):
+        assert lib.mla_output_projection_workspace_size(B, dim) == 0
+    # the fused call holds the decode scratch, the per-head outputs and the partials
+    for B, K in ((64, 2048), (3, 100)):
+        dec = lib.mla_sparse_decode_workspace_size(B, K, 4096)
+        proj = lib.mla_output_projection_workspace_size(B, 7168)
+        need = dec + B * 16384 * 2 + proj
+        got = lib.mla_sparse_decode_project_workspace_size(B, K, 4096, 7168)
+        assert need <= got <= need + 3 * 256
+    assert lib.mla_sparse_decode_project_workspace_size(1, 1, 1, 100) == 0
+    assert lib.mla_sparse_decode_project_workspace_size(0, 1, 1, 7168) == 0
+
+
+def test_projection_rejects_bad_arguments_without_a_launch(lib):
+    A = 0x10000
+    ok = dict(x=_fake(A), wo=_fake(A), delta=_fake(A), B=4, dim=7168, ws=_fake(A), wsb=1 << 30, st=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.mla_output_projection(a["x"], a["wo"], a["delta"], a["B"], a["dim"], a["ws"], a["wsb"], a["st"],
+                                         None)
+
+    for name in ("x", "wo", "delta"):
+        assert call(**{name: None}) == INVALID_ARG
+        assert call(**{name: _fake(A + 8)}) == INVALID_ARG
+    for dim in (0, 64, 100, 7168 + 64, 1 << 17):
+        assert call(dim=dim) == INVALID_ARG
+    assert call(B=0) == INVALID_ARG
+    assert call(st=_fake(A + 2)) == INVALID_ARG
+
+    args = [_fake(A)] * 7
+    base = dict(wo=_fake(A), delta=_fake(A), B=2, K=16, S=32, dim=7168, scale=0.07)
+
+    def call_p(ptrs=None, **kw):
+        a = dict(base, **kw)
+        p = ptrs or args
+        return lib.mla_sparse_decode_project(*p[:7], ctypes.c_float(a["scale"]), a["wo"], a["delta"], a["B"], a["K"],
+                                             a["S"], a["dim"], _fake(A), 1 << 30, None, None, None)
+
+    for i in range(7):
+        bad = list(args)
+        bad[i] = None
+        assert call_p(bad) == INVALID_ARG
+    assert call_p(wo=None) == INVALID_ARG
+    assert call_p(delta=_fake(A + 4)) == INVALID_ARG
+    assert call_p(dim=100) == INVALID_ARG
+    assert call_p(K=0) == INVALID_ARG
+    assert call_p(scale=float("nan")) == INVALID_ARG

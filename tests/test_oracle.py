@@ -12,6 +12,9 @@ the pages and the mathematics fix:
       excerpt's einsums run literally in torch float64;
   plus closed forms (one selected key; zero query) and set semantics of the
   index list (order, duplicates, padding).
+The output projection (page "Attention update") is pinned by a hand-derived
+case, basis vectors (a unit input picks one column of wo), linearity, BLAS
+float64 matmul, and the page's ``wo(x.flatten(2))`` in torch float64.
 """
 import itertools
 import json
@@ -23,7 +26,7 @@ import pytest
 import torch
 
 import oracle
-from tests.oracle_refs import nonabsorbed, transcript, to_f64, valid_set
+from tests.oracle_refs import nonabsorbed, transcript, transcript_projection, to_f64, valid_set
 from sparse_latent_attention_absorb_b200 import workloads as wl
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -315,6 +318,10 @@ def test_page_shapes_fixture():
     assert g["kv_latent"] == wl.D_LAT and g["value"] == wl.D_V
     assert g["cached_positions_example"] == wl.WORKLOADS["b1_ctx1001_top256"].end_pos[0]
     assert wl.SCALE == pytest.approx(g["content_plus_rotary"] ** -0.5, rel=1e-7)
+    assert g["model_width"] == wl.D_MODEL
+    assert g["wo_inputs"] == g["heads"] * g["value"] == wl.H * wl.D_V
+    d = wl.generate_projection(2, dim=256)
+    assert tuple(d["x"].shape) == (2, g["wo_inputs"]) and tuple(d["wo"].shape) == (256, g["wo_inputs"])
 
 
 def test_regression_fixture():
@@ -328,3 +335,60 @@ def test_regression_fixture():
     res = run(case)
     np.testing.assert_allclose(res.out.reshape(-1), np.array(g["out"]), rtol=1e-13, atol=1e-15)
     np.testing.assert_allclose(res.lse.reshape(-1), np.array(g["lse"]), rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------- output projection
+
+def test_projection_hand_derived():
+    x = np.array([[1.0, 2.0, 3.0], [0.5, -1.0, 0.0]])
+    wo = np.array([[1.0, 0.0, 0.0], [0.0, 1.0, 1.0], [2.0, -1.0, 0.5]])
+    # row 0: (1, 2 + 3, 2 - 2 + 1.5); row 1: (0.5, -1, 1 + 1 + 0)
+    np.testing.assert_array_equal(oracle.output_projection(x, wo), [[1.0, 5.0, 1.5], [0.5, -1.0, 2.0]])
+
+
+def test_projection_unit_inputs_pick_columns_of_wo():
+    rng = np.random.default_rng(11)
+    n_in, dim = 64, 40
+    wo = rng.standard_normal((dim, n_in))
+    ks = [0, 7, 31, 63]
+    x = np.zeros((len(ks), n_in))
+    for r, k in enumerate(ks):
+        x[r, k] = 1.0
+    got = oracle.output_projection(x, wo)
+    for r, k in enumerate(ks):
+        np.testing.assert_array_equal(got[r], wo[:, k])
+
+
+def test_projection_is_linear():
+    rng = np.random.default_rng(12)
+    n_in, dim = 96, 33
+    wo = rng.standard_normal((dim, n_in))
+    x1, x2 = rng.standard_normal((3, n_in)), rng.standard_normal((3, n_in))
+    a = 0.75
+    lhs = oracle.output_projection(a * x1 + x2, wo)
+    rhs = a * oracle.output_projection(x1, wo) + oracle.output_projection(x2, wo)
+    assert rel_err(lhs, rhs) < 1e-13
+
+
+def test_projection_matches_blas_and_page_transcript_at_real_width():
+    """bf16 inputs of the real shapes (x [B,128,128] flattened per row, wo
+    [dim,16384]), widened exactly: BLAS float64 matmul and the page's
+    wo(x.flatten(2)) agree with the oracle."""
+    d = wl.generate_projection(3, dim=256, seed=17)
+    x3 = d["x"].view(3, wl.H, wl.D_V)
+    got = oracle.output_projection(x3, d["wo"])
+    blas = to_f64(d["x"]) @ to_f64(d["wo"]).T
+    assert rel_err(got, blas) < 1e-12
+    assert rel_err(got, transcript_projection(x3, d["wo"])) < 1e-12
+    # the flattening is per row, head-major: k = 128 h + e
+    assert got[1, 5] == pytest.approx(float(sum(to_f64(x3)[1, h, e] * to_f64(d["wo"])[5, 128 * h + e]
+                                                for h in range(wl.H) for e in range(wl.D_V))), rel=1e-12)
+
+
+def test_projection_row_subset_matches_full_run():
+    d = wl.generate_projection(5, dim=128, seed=18)
+    full = oracle.output_projection(d["x"], d["wo"])
+    part = oracle.output_projection(d["x"], d["wo"], rows=[4, 0])
+    np.testing.assert_array_equal(part, full[[4, 0]])
+    with pytest.raises(RuntimeError):
+        oracle.output_projection(d["x"], d["wo"], rows=[5])

@@ -330,3 +330,63 @@ def test_online_softmax_rescales_when_scores_grow_along_the_tiles():
     assert np.all(np.isfinite(got))
     assert np.max(np.abs(got - ref.out)) <= out_bound(ref.out)
     assert np.max(np.abs(lse.double().cpu().numpy()[rows] - ref.lse)) <= 1e-2
+
+
+# ------------------------------------------------------------------ output projection (page "Attention update")
+
+def proj_bound(ref):
+    """bf16 of an fp32 sum: one bf16 rounding (half an ulp is 2^-9 relative;
+    2^-8 allowed) plus fp32 accumulation over 16384 products in an order the
+    oracle does not fix (bounded by 1e-4 of the largest output)."""
+    return 2.0 ** -8 * np.abs(ref) + 1e-4 * float(np.max(np.abs(ref)))
+
+
+@pytest.mark.parametrize("B,dim", [(1, 128), (3, 384), (17, 1024), (64, 7168), (100, 2048), (300, 256),
+                                   (1000, 7168)])
+def test_output_projection_matches_oracle(B, dim):
+    """delta = x . wo^T.  Covers: fewer tiles than SMs (work split unit by
+    unit, partials reduced in a fixed order; B=1, dim=128 spreads one tile
+    over all SMs), two batch tiles (B=300), and one CTA per tile writing
+    bf16 directly (B=1000 at the pages' width: 4 x 56 tiles)."""
+    d = wl.generate_projection(B, dim, seed=3000 + B)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    delta = pkg.mla_output_projection(d["x"].to(DEV), d["wo"].to(DEV), d_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rows = list(range(B)) if B <= 17 else sorted({0, 1, B // 2, B - 2, B - 1})
+    ref = oracle.output_projection(d["x"], d["wo"], rows=rows)
+    got = delta.double().cpu().numpy()[rows]
+    assert np.all(np.abs(got - ref) <= proj_bound(ref))
+
+
+def test_output_projection_is_deterministic():
+    d = wl.generate_projection(64, 1024, seed=3100)
+    x, wo = d["x"].to(DEV), d["wo"].to(DEV)
+    a = pkg.mla_output_projection(x, wo)
+    b = pkg.mla_output_projection(x, wo)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name", ["small_b5_ctx40-700_top333", "b1_ctx1001_top256"])
+def test_decode_project_matches_oracle_chain(name):
+    """The fused call equals the two separate calls bit for bit, and the
+    oracle's decode followed by its projection within the decode step's
+    tolerance (the decode's rounding passes through wo, whose rows have unit
+    norm)."""
+    d = wl.generate(name)
+    g = to_dev(d)
+    B = d["q_nope"].shape[0]
+    wo_cpu = wl.generate_projection(1, wl.D_MODEL, seed=3200)["wo"]
+    wo = wo_cpu.to(DEV)
+    delta = pkg.mla_sparse_decode_project(g["q_nope"], g["q_pe"], g["kv_cache"], g["pe_cache"], g["end_pos"],
+                                          g["topk_idx"], g["wkv_b"], g["scale"], wo)
+    out, _ = gpu_decode(g, lse=False)
+    delta2 = pkg.mla_output_projection(out, wo)
+    torch.cuda.synchronize()
+    assert torch.equal(delta, delta2)
+    ref_out = run_oracle(d).out                                   # fp64 [B, 128, 128]
+    ref = oracle.output_projection(ref_out, wo_cpu.double().numpy())
+    got = delta.double().cpu().numpy()
+    assert got.shape == (B, wl.D_MODEL)
+    assert np.max(np.abs(got - ref)) <= out_bound(ref)
