@@ -304,7 +304,8 @@ int launch_projection(const void* x, const void* wo, void* delta, int B, int dim
     return rc;
   if (p.direct) return MLA_OK;
   dim3 grid((unsigned)p.tiles, ceil_div(p.n_tile, kProjReduceRows));
-  return launch_ex(projection_reduce_kernel, grid, dim3(kProjM), 0, stream, true, static_cast<const float*>(partial),
+  return launch_ex(projection_reduce_kernel, grid, dim3(kProjReduceThreads), 0, stream, true,
+                   static_cast<const float*>(partial),
                    static_cast<__nv_bfloat16*>(delta), B, dim, p.n_tile, p.n_ctas);
 }
 

@@ -230,32 +230,42 @@ projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_consta
 }
 
 // delta[b, 128 m + n] = bf16( sum over the CTAs c whose units cover the tile
-// (y, m), in increasing c, of their partial for it ).  Grid (tiles, row groups
-// of kProjReduceRows within a tile); thread n = wo row within the tile.
-__global__ void __launch_bounds__(kProjM)
+// (y, m), in increasing c, of their partial for it ).  Grid (tiles, groups of
+// kProjReduceRows rows of a tile); thread t sums row t / 32 of its group,
+// wo rows 4 (t % 32) .. +3, with one independent 16-byte load per
+// contributing CTA.  Only the split mode launches it: fewer tiles than SMs,
+// so unit and CTA indices stay far below 2^31 and 32-bit arithmetic is exact.
+constexpr int kProjReduceThreads = kProjReduceRows * 32;
+
+__global__ void __launch_bounds__(kProjReduceThreads)
 projection_reduce_kernel(const float* __restrict__ partial, __nv_bfloat16* __restrict__ delta, int B, int dim,
                          int n_tile, int n_ctas) {
   const int t = blockIdx.x;
   const int m_tiles = dim / kProjM;
   const int m = t % m_tiles;
   const int row0 = (t / m_tiles) * n_tile;
-  const int j0 = blockIdx.y * kProjReduceRows;  // first row of this CTA within the tile
-  const int n = threadIdx.x;
-  const long long U = (long long)m_tiles * ((B + n_tile - 1) / n_tile) * kProjKBlocks;
-  const long long first_unit = (long long)t * kProjKBlocks;
-  const int c_lo = proj_cta_of_unit(first_unit, U, n_ctas);
-  const int c_hi = proj_cta_of_unit(first_unit + kProjKBlocks - 1, U, n_ctas);
+  const int j = blockIdx.y * kProjReduceRows + (int)(threadIdx.x >> 5);  // row within the tile
+  const int n4 = (int)(threadIdx.x & 31) * 4;
+  const int U = m_tiles * ((B + n_tile - 1) / n_tile) * kProjKBlocks;
+  const int first_unit = t * kProjKBlocks;
+  const int c_lo = ((first_unit + 1) * n_ctas - 1) / U;              // CTA holding the tile's first unit
+  const int c_hi = ((first_unit + kProjKBlocks) * n_ctas - 1) / U;   // ... and its last
   grid_dep_wait();  // the partials come from projection_kernel
-  for (int r = 0; r < kProjReduceRows; ++r) {
-    const int j = j0 + r;
-    if (j >= n_tile || row0 + j >= B) break;
-    float acc = 0.f;
-    for (int cc = c_lo; cc <= c_hi; ++cc) {
-      const int seg = (proj_unit_begin(cc, U, n_ctas) / kProjKBlocks == t) ? 0 : 1;
-      acc += __ldg(partial + ((size_t)(2 * cc + seg) * n_tile + j) * kProjM + n);
-    }
-    delta[(size_t)(row0 + j) * dim + (size_t)m * kProjM + n] = __float2bfloat16_rn(acc);
+  if (j >= n_tile || row0 + j >= B) return;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int cc = c_lo; cc <= c_hi; ++cc) {
+    const int seg = (cc * U / n_ctas) / kProjKBlocks == t ? 0 : 1;  // the tile is cc's first or second segment
+    const float4 v = __ldg(reinterpret_cast<const float4*>(partial + ((size_t)(2 * cc + seg) * n_tile + j) * kProjM + n4));
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
   }
+  uint2 packed;
+  packed.x = pack_bf16x2(acc.x, acc.y);
+  packed.y = pack_bf16x2(acc.z, acc.w);
+  *reinterpret_cast<uint2*>(delta + (size_t)(row0 + j) * dim + (size_t)m * kProjM + n4) = packed;
 }
 
 }  // namespace mla
