@@ -370,6 +370,25 @@ def gpu_arm(args, rank, world, device):
     p_bytes = p_dim * 16384 * 2 + B * 16384 * 2 + B * p_dim * 2
     del p_wo
 
+    # ---- the sparse prefill (page "Queries", prefill mode): one sequence of
+    # 4096 positions, top-2048, one row per query position reading the
+    # chunk's own latents (4.7 MB: they stay in L2)
+    pf = wl.generate_prefill(1, 4096, 2048, seed=5101)
+    pf_sel = int(((pf["topk_idx"] >= 0) & (pf["topk_idx"] < pf["end_pos"].unsqueeze(1))).sum())
+    pfd = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in pf.items()}
+    R_pf, K_pf, S_pf = pf["q_nope"].shape[0], pf["topk_idx"].shape[1], pf["kv_cache"].shape[1]
+    pf_out = torch.empty((R_pf, 128, 128), dtype=torch.bfloat16, device=device)
+    pf_ws = torch.empty(lib.mla_sparse_decode_workspace_size(R_pf, K_pf, S_pf), dtype=torch.uint8, device=device)
+
+    def k_prefill(i):
+        return lib.mla_sparse_prefill(P(pfd["q_nope"]), P(pfd["q_pe"]), P(pfd["kv_cache"]), P(pfd["pe_cache"]),
+                                      P(pfd["cache_slot"]), P(pfd["end_pos"]), P(pfd["topk_idx"]), P(pfd["wkv_b"]),
+                                      ctypes.c_float(pfd["scale"]), P(pf_out), R_pf, K_pf, S_pf, 1, P(pf_ws),
+                                      pf_ws.numel(), None, None, sv)
+
+    t_prefill = time_kernel(k_prefill, 5)
+    del pfd, pf_out, pf_ws
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if rank == 0 or world > 1:
@@ -457,6 +476,10 @@ def gpu_arm(args, rank, world, device):
                        "roofline": {"bound": "hbm", "achieved": p_bytes / (t_project * 1e-3) / 1e9, "peak": hbm,
                                     "unit": "GB/s", "frac": p_bytes / (t_project * 1e-3) / 1e9 / hbm,
                                     "alg_bytes_per_call": p_bytes, "peak_source": f"{kind} hbm_gbs"}},
+        "prefill": {"what": "sparse prefill of one 4096-position sequence, top-2048, causal: one row per query "
+                            "position (mla_sparse_prefill)", "ms_per_call": t_prefill,
+                    "tokens_per_s": R_pf / (t_prefill * 1e-3), "selected_positions": pf_sel,
+                    "gathered_GBps": pf_sel * 1152 / (t_prefill * 1e-3) / 1e9},
         "gpu_launches": launches,
         "e2e": e2e,
         "clocks": clocks.summary(),

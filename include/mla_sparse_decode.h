@@ -209,6 +209,37 @@ int mla_sparse_decode_host(const void* h_q_nope, const void* h_q_pe, const int32
                            size_t workspace_bytes, float* lse_out, int* d_status, cudaStream_t stream);
 
 /*
+ * Sparse prefill (the "MHA prefill" branch, model.py 574-589, as shown on the
+ * atlas page "Queries" in prefill mode): every query position s of a
+ * sequence attends to the positions t of the same sequence that the indexer
+ * selected for it and that the causal mask allows (t <= s):
+ *   x[b,s,h,:] = sum_t softmax_t( scale * q[b,s,h] . k[b,t,h] ) v[b,t,h]
+ * with k = [W_UK c_t ; k^R_t] and v = W_UV c_t.  The pages up-project every
+ * latent into per-head keys and values; this entry point computes the same
+ * result in the absorbed form of mla_sparse_decode (q . k = (q_nope W_UK) .
+ * c_t + q_pe . k^R_t, and the mix of W_UV c_t is W_UV applied to the mix of
+ * c_t), so a selected position costs one 1152-byte latent + rotary row
+ * instead of 128 heads' keys and values.
+ * Each of the R rows is one query position:
+ *   q_nope, q_pe, out, lse_out, topk_idx  as in mla_sparse_decode with B = R
+ *   kv_cache bf16 [n_slots,S_max,512], pe_cache bf16 [n_slots,S_max,64]: the
+ *            latents of n_slots sequences (a prefill chunk: S_max = seqlen)
+ *   cache_slot int32 [R]  the sequence of each row (16-byte aligned); a
+ *            value outside [0, n_slots) gives the row no valid position
+ *   end_pos  int32 [R]    the causal bound: s + 1 for the query at position s
+ *            (positions t >= end_pos[r] are masked, as the causal mask does)
+ *   workspace: mla_sparse_decode_workspace_size(R, K, S_max) bytes
+ * For the pages' prefill of B sequences of seqlen positions:
+ * R = B * seqlen, cache_slot[b*seqlen + s] = b, end_pos[b*seqlen + s] = s+1,
+ * topk_idx[b*seqlen + s] = the indexer's selection for position s.
+ * Returns an mla_status.
+ */
+int mla_sparse_prefill(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                       const int32_t* cache_slot, const int32_t* end_pos, const int32_t* topk_idx, const void* wkv_b,
+                       float scale, void* out, int R, int K, int S_max, int n_slots, void* workspace,
+                       size_t workspace_bytes, float* lse_out, int* d_status, cudaStream_t stream);
+
+/*
  * Output projection (model.py 607-608 as shown on the atlas page "Attention
  * update": the head outputs of a row are flattened and projected back to the
  * model width by wo, a RowParallelLinear from 128*128 inputs to dim outputs;

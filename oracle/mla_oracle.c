@@ -87,6 +87,14 @@ static int selected_positions(const int32_t *idx_row, int K, int end_pos,
  * The decode step for the batch rows listed in `rows` (n_rows entries; each a
  * batch index in [0, B)).  Output r corresponds to batch row rows[r].
  *
+ * Row b reads the cached latents and rotary keys of slot cache_slot[b] when
+ * cache_slot is given (kv [n_slots, S_max, Dl], pe [n_slots, S_max, Dr]),
+ * else of slot b (n_slots = B).  With one row per query position of a
+ * sequence, a slot per sequence and end_pos = s + 1 (the causal bound), this
+ * is the "MHA prefill" branch of the page "Queries" (model.py 574-589) in
+ * absorbed form: a row whose slot is outside [0, n_slots) has no valid
+ * position.
+ *
  * Outputs (any optional one may be NULL):
  *   out    [n_rows, H, Dv]      required
  *   lse    [n_rows, H]          log sum_{t in T_b} exp(s[t])  (natural log)
@@ -101,7 +109,7 @@ int oracle_mla_sparse_decode_f64(
     const void *wkv_b, int in_bf16,
     const int32_t *end_pos, const int32_t *topk_idx, double scale,
     int B, int K, int S_max, int H, int Dn, int Dr, int Dl, int Dv,
-    const int32_t *rows, int n_rows,
+    const int32_t *rows, int n_rows, const int32_t *cache_slot, int n_slots,
     double *out, double *lse, double *q_lat, double *o_lat, double *w_full)
 {
     if (B < 0 || K < 0 || S_max < 0 || H <= 0 || Dn <= 0 || Dr < 0 ||
@@ -121,6 +129,8 @@ int oracle_mla_sparse_decode_f64(
         int ep = end_pos[b];
         if (ep > S_max)
             ep = S_max; /* positions past the cache do not exist */
+        if (cache_slot && (cache_slot[b] < 0 || cache_slot[b] >= n_slots))
+            ep = 0;     /* no such sequence: nothing is selected */
         sel[r] = (int32_t *)malloc(sizeof(int32_t) * ((size_t)(ep > 0 ? ep : 0) + 1));
         if (sel[r] == NULL) {
             fail = 1;
@@ -137,6 +147,7 @@ int oracle_mla_sparse_decode_f64(
             for (int h = 0; h < H; ++h) {
                 const int b = rows[r];
                 const int n = nsel[r];
+                const size_t slot = cache_slot ? (size_t)(n > 0 ? cache_slot[b] : 0) : (size_t)b;
                 const int32_t *T = sel[r];
                 double *ql = (double *)malloc(sizeof(double) * (size_t)Dl);
                 double *ol = (double *)malloc(sizeof(double) * (size_t)Dl);
@@ -165,8 +176,8 @@ int oracle_mla_sparse_decode_f64(
                 double m = -INFINITY;
                 for (int j = 0; j < n; ++j) {
                     int t = T[j];
-                    size_t kvrow = ((size_t)b * S_max + t) * Dl;
-                    size_t perow = ((size_t)b * S_max + t) * Dr;
+                    size_t kvrow = (slot * S_max + t) * Dl;
+                    size_t perow = (slot * S_max + t) * Dr;
                     double acc_lat = 0.0, acc_rope = 0.0;
                     for (int c = 0; c < Dl; ++c)
                         acc_lat += ql[c] * load_elem(kv, kvrow + c, in_bf16);
@@ -191,7 +202,7 @@ int oracle_mla_sparse_decode_f64(
                 for (int c = 0; c < Dl; ++c)
                     ol[c] = 0.0;
                 for (int j = 0; j < n; ++j) {
-                    size_t kvrow = ((size_t)b * S_max + T[j]) * Dl;
+                    size_t kvrow = (slot * S_max + T[j]) * Dl;
                     for (int c = 0; c < Dl; ++c)
                         ol[c] += w[j] * load_elem(kv, kvrow + c, in_bf16);
                 }

@@ -53,6 +53,7 @@ def _load():
             p, p, ctypes.c_double,       # end_pos topk_idx scale
             i, i, i, i, i, i, i, i,      # B K S_max H Dn Dr Dl Dv
             p, i,                        # rows n_rows
+            p, i,                        # cache_slot n_slots
             p, p, p, p, p,               # out lse q_lat o_lat w_full
         ]
         lib.oracle_output_projection_f64.restype = ctypes.c_int
@@ -113,7 +114,7 @@ class OracleResult:
 
 
 def mla_sparse_decode(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx,
-                      wkv_b, scale, rows=None, *, want_q_lat=False,
+                      wkv_b, scale, rows=None, *, cache_slot=None, want_q_lat=False,
                       want_o_lat=False, want_weights=False) -> OracleResult:
     """Run the oracle on the given inputs.
 
@@ -125,6 +126,10 @@ def mla_sparse_decode(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx,
     3-D, in which case Dv = wkv_b.shape[1] - Dn.
 
     ``rows`` selects batch rows (default: all); result r is batch row rows[r].
+    ``cache_slot`` [B] (optional): row b reads kv_cache[cache_slot[b]] and
+    pe_cache[cache_slot[b]] (the caches then hold n_slots = kv_cache.shape[0]
+    sequences); the prefill of the page "Queries" is one row per query
+    position with end_pos = position + 1.
     """
     import numbers
     try:
@@ -154,6 +159,10 @@ def mla_sparse_decode(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx,
     ti = _ints(topk_idx)
     rows_a = _ints(np.arange(B) if rows is None else rows).reshape(-1)
     n = int(rows_a.shape[0])
+    slots = None if cache_slot is None else _ints(cache_slot).reshape(-1)
+    n_slots = int(kv_cache.shape[0])
+    if slots is not None:
+        assert slots.shape[0] == B, "cache_slot must hold one slot per row"
 
     out = np.zeros((n, H, Dv), np.float64)
     lse = np.zeros((n, H), np.float64)
@@ -165,7 +174,7 @@ def mla_sparse_decode(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx,
         _ptr(qn), _ptr(qp), _ptr(kv), _ptr(pe), _ptr(wb), int(is_bf16),
         _ptr(ep), _ptr(ti), float(scale),
         B, K, S_max, H, Dn, Dr, Dl, Dv,
-        _ptr(rows_a), n,
+        _ptr(rows_a), n, _ptr(slots), n_slots,
         _ptr(out), _ptr(lse), _ptr(ql), _ptr(ol), _ptr(wf))
     if rc != 0:
         raise RuntimeError(f"oracle failed with code {rc}")

@@ -9,10 +9,10 @@ The CUDA library is loaded on first use and its absence is an error.
 """
 from .binding import (MLAError, host_workspace_size, load_library, mla_absorb_q, mla_combine_value_up,
                       mla_output_projection, mla_sparse_attend, mla_sparse_decode, mla_sparse_decode_host,
-                      mla_sparse_decode_project, num_splits, project_workspace_size, projection_workspace_size,
+                      mla_sparse_decode_project, mla_sparse_prefill, num_splits, project_workspace_size, projection_workspace_size,
                       workspace_size)
 
 __all__ = ["MLAError", "host_workspace_size", "load_library", "mla_absorb_q", "mla_combine_value_up",
            "mla_output_projection", "mla_sparse_attend", "mla_sparse_decode", "mla_sparse_decode_host",
-           "mla_sparse_decode_project", "num_splits", "project_workspace_size", "projection_workspace_size",
+           "mla_sparse_decode_project", "mla_sparse_prefill", "num_splits", "project_workspace_size", "projection_workspace_size",
            "workspace_size"]

@@ -26,7 +26,7 @@ EXPORTS = ("mla_status_string", "mla_num_splits", "mla_sparse_decode_workspace_s
            "mla_absorb_q", "mla_sparse_attend", "mla_combine_value_up", "mla_sparse_decode_noalloc",
            "mla_sparse_decode_host_workspace_size", "mla_sparse_decode_host",
            "mla_output_projection_workspace_size", "mla_output_projection",
-           "mla_sparse_decode_project_workspace_size", "mla_sparse_decode_project")
+           "mla_sparse_decode_project_workspace_size", "mla_sparse_decode_project", "mla_sparse_prefill")
 STATIC_SCRATCH_BYTES = 32 << 20  # MLA_STATIC_SCRATCH_BYTES
 
 _lib = None
@@ -75,6 +75,8 @@ def load_library():
     lib.mla_sparse_decode_project_workspace_size.argtypes = [i, i, i, i]
     lib.mla_sparse_decode_project.restype = i
     lib.mla_sparse_decode_project.argtypes = [p, p, p, p, p, p, p, f, p, p, i, i, i, i, p, sz, p, p, p]
+    lib.mla_sparse_prefill.restype = i
+    lib.mla_sparse_prefill.argtypes = [p, p, p, p, p, p, p, p, f, p, i, i, i, i, p, sz, p, p, p]
     _lib = lib
     return lib
 
@@ -361,3 +363,38 @@ def mla_sparse_decode_project(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_id
                                        _ptr(d_status), _stream(stream))
     _raise(rc, "mla_sparse_decode_project")
     return delta
+
+
+def mla_sparse_prefill(q_nope, q_pe, kv_cache, pe_cache, cache_slot, end_pos, topk_idx, wkv_b, scale, out=None,
+                       workspace=None, lse_out=None, d_status=None, stream=None):
+    """Sparse prefill: one row per query position; row r reads the latents of
+    sequence cache_slot[r] (kv_cache [n_slots, S_max, 512]) up to its causal
+    bound end_pos[r].  Returns ``out`` (bf16 [R,128,128])."""
+    lib = load_library()
+    R, K = q_nope.shape[0], topk_idx.shape[1]
+    n_slots, S_max = kv_cache.shape[0], kv_cache.shape[1]
+    bf = torch.bfloat16
+    _check(q_nope, "q_nope", bf, (R, H, D_NOPE))
+    _check(q_pe, "q_pe", bf, (R, H, D_ROPE))
+    _check(kv_cache, "kv_cache", bf, (n_slots, S_max, D_LAT))
+    _check(pe_cache, "pe_cache", bf, (n_slots, S_max, D_ROPE))
+    _check(cache_slot, "cache_slot", torch.int32, (R,))
+    _check(end_pos, "end_pos", torch.int32, (R,))
+    _check(topk_idx, "topk_idx", torch.int32, (R, K))
+    _check(wkv_b, "wkv_b", bf, (H * (D_NOPE + D_V), D_LAT))
+    if out is None:
+        out = torch.empty((R, H, D_V), dtype=bf, device=q_nope.device)
+    _check(out, "out", bf, (R, H, D_V))
+    if lse_out is not None:
+        _check(lse_out, "lse_out", torch.float32, (R, H))
+    if d_status is not None:
+        _check(d_status, "d_status", torch.int32, (1,))
+    if workspace is None:
+        workspace = torch.empty(workspace_size(R, K, S_max), dtype=torch.uint8, device=q_nope.device)
+    _check(workspace, "workspace", torch.uint8)
+    rc = lib.mla_sparse_prefill(_ptr(q_nope), _ptr(q_pe), _ptr(kv_cache), _ptr(pe_cache), _ptr(cache_slot),
+                                _ptr(end_pos), _ptr(topk_idx), _ptr(wkv_b), float(scale), _ptr(out), R, K, S_max,
+                                n_slots, _ptr(workspace), workspace.numel(), _ptr(lse_out), _ptr(d_status),
+                                _stream(stream))
+    _raise(rc, "mla_sparse_prefill")
+    return out

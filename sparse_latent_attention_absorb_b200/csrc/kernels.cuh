@@ -313,7 +313,8 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
                      const __nv_bfloat16* __restrict__ kv_cache, const __nv_bfloat16* __restrict__ pe_cache,
                      const int32_t* __restrict__ end_pos, const int32_t* __restrict__ topk_idx, float scale,
                      void* __restrict__ o_part, float* __restrict__ lse_part, int K, int S_max, int n_split,
-                     int span, const __nv_bfloat16* __restrict__ w_next, int* d_status) {
+                     int span, const __nv_bfloat16* __restrict__ w_next, const int32_t* __restrict__ cache_slot,
+                     int n_slots, int* d_status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -327,6 +328,17 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
   const int n_tiles = k_end > k_begin ? (k_end - k_begin + kNt - 1) / kNt : 0;
   int ep = end_pos[b];
   ep = ep < 0 ? 0 : (ep > S_max ? S_max : ep);
+  // Cache slot of row b: b itself (decode), or cache_slot[b] when rows are
+  // query positions sharing a sequence's latents (prefill).  A slot outside
+  // [0, n_slots) leaves the row with no valid position (nothing is read).
+  int slot = b;
+  if (cache_slot != nullptr) {
+    slot = cache_slot[b];
+    if (slot < 0 || slot >= n_slots) {
+      slot = 0;
+      ep = 0;
+    }
+  }
   const int32_t* idx_row = topk_idx + (size_t)b * K;
 
   const uint32_t sStage = smem_u32(smem + kOffStage);
@@ -382,8 +394,8 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     // successive waits on one stage's kv_empty are exactly one phase apart.
     const int g = warp - kGatherWarp0;
     const int row0 = 16 * g;
-    const __nv_bfloat16* kv_row0 = kv_cache + (size_t)b * S_max * kDl + rank * 256;
-    const __nv_bfloat16* pe_row0 = pe_cache + (size_t)b * S_max * kDr + rank * 32;
+    const __nv_bfloat16* kv_row0 = kv_cache + (size_t)slot * S_max * kDl + rank * 256;
+    const __nv_bfloat16* pe_row0 = pe_cache + (size_t)slot * S_max * kDr + rank * 32;
     // Index of row 16g + (lane % 16) of tile 2p + lane / 16 (a pair of tiles
     // per register), or -1 for a padding or out-of-range slot.
     auto load_pair = [&](int pr) -> int {

@@ -262,14 +262,14 @@ int launch_absorb(const void* q_nope, const void* wkv_b, void* q_lat, int B, int
 int launch_attend(const void* q_lat, const void* q_pe, const void* kv_cache, const void* pe_cache,
                   const int32_t* end_pos, const int32_t* topk_idx, float scale, void* o_part, float* lse_part, int B,
                   int K, int S_max, int n_split, int span, const void* w_next, int* d_status, cudaStream_t stream,
-                  bool pdl) {
+                  bool pdl, const int32_t* cache_slot = nullptr, int n_slots = 0) {
   const long long ctas = 2LL * B * n_split;
   if (ctas > 0x7fffffffLL) return MLA_ERR_INVALID_ARG;
   return launch_ex(sparse_attend_kernel, dim3((unsigned)ctas), dim3(kAttendThreads), kAttendSmemBytes, stream, pdl,
                    static_cast<const __nv_bfloat16*>(q_lat), static_cast<const __nv_bfloat16*>(q_pe),
                    static_cast<const __nv_bfloat16*>(kv_cache), static_cast<const __nv_bfloat16*>(pe_cache), end_pos,
                    topk_idx, scale, o_part, lse_part, K, S_max, n_split, span,
-                   static_cast<const __nv_bfloat16*>(w_next), d_status);
+                   static_cast<const __nv_bfloat16*>(w_next), cache_slot, n_slots, d_status);
 }
 
 int launch_combine(const void* o_part, const float* lse_part, const void* wkv_b, void* out, float* lse_out, int B,
@@ -408,10 +408,15 @@ extern "C" int mla_combine_value_up(const void* o_part, const float* lse_part, c
   return launch_combine(o_part, lse_part, wkv_b, out, lse_out, B, n_split, nullptr, stream, false);
 }
 
-extern "C" int mla_sparse_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
-                                 const int32_t* end_pos, const int32_t* topk_idx, const void* wkv_b, float scale,
-                                 void* out, int B, int K, int S_max, void* workspace, size_t workspace_bytes,
-                                 float* lse_out, int* d_status, cudaStream_t stream) {
+namespace {
+// The three kernels over B rows: row b is one query (its q_nope, q_pe, index
+// row and end position) and reads cache slot cache_slot[b], or b when
+// cache_slot is null.  Shared by the decode step (a row per batch row) and
+// the prefill (a row per query position of a sequence).
+int run_rows(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+             const int32_t* end_pos, const int32_t* topk_idx, const void* wkv_b, float scale, void* out, int B, int K,
+             int S_max, const int32_t* cache_slot, int n_slots, void* workspace, size_t workspace_bytes,
+             float* lse_out, int* d_status, cudaStream_t stream) {
   const void* ptrs[] = {q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, out};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return MLA_ERR_INVALID_ARG;
@@ -440,9 +445,30 @@ extern "C" int mla_sparse_decode(const void* q_nope, const void* q_pe, const voi
   // The attention kernel also pulls W_UV into L2 near its end, for the
   // value-up kernel.
   if ((rc = launch_attend(q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, scale, o_part, lse_part, B, K, S_max,
-                          n_split, span, wkv_b, d_status, stream, true)) != MLA_OK)
+                          n_split, span, wkv_b, d_status, stream, true, cache_slot, n_slots)) != MLA_OK)
     return rc;
   return launch_combine(o_part, lse_part, wkv_b, out, lse_out, B, n_split, d_status, stream, true);
+}
+}  // namespace
+
+extern "C" int mla_sparse_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                                 const int32_t* end_pos, const int32_t* topk_idx, const void* wkv_b, float scale,
+                                 void* out, int B, int K, int S_max, void* workspace, size_t workspace_bytes,
+                                 float* lse_out, int* d_status, cudaStream_t stream) {
+  return run_rows(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, scale, out, B, K, S_max, nullptr, B,
+                  workspace, workspace_bytes, lse_out, d_status, stream);
+}
+
+// The sparse prefill (see the header): R query rows over n_slots sequences'
+// latents, row r reading slot cache_slot[r] with its own causal end position.
+extern "C" int mla_sparse_prefill(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                                  const int32_t* cache_slot, const int32_t* end_pos, const int32_t* topk_idx,
+                                  const void* wkv_b, float scale, void* out, int R, int K, int S_max, int n_slots,
+                                  void* workspace, size_t workspace_bytes, float* lse_out, int* d_status,
+                                  cudaStream_t stream) {
+  if (!cache_slot || !aligned16(cache_slot) || n_slots < 1) return MLA_ERR_INVALID_ARG;
+  return run_rows(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, scale, out, R, K, S_max, cache_slot,
+                  n_slots, workspace, workspace_bytes, lse_out, d_status, stream);
 }
 
 #ifdef MLA_TRACE

@@ -200,3 +200,36 @@ def generate_projection(B: int, dim: int = D_MODEL, seed: int = 2001) -> dict:
         "x": _bf16_normal((B, n_in), gen),
         "wo": _bf16_normal((dim, n_in), gen, std=n_in ** -0.5, chunk_dim0=dim * n_in > (1 << 26)),
     }
+
+
+def generate_prefill(B: int, seqlen: int, K: int, seed: int = 2101) -> dict:
+    """Inputs of one sparse prefill (page "Queries", prefill mode), on the CPU,
+    one row per query position: q_nope [B*seqlen,128,128], q_pe
+    [B*seqlen,128,64], kv_cache [B,seqlen,512], pe_cache [B,seqlen,64] (bf16;
+    the chunk's own latents), cache_slot, end_pos and topk_idx [B*seqlen, K]
+    (int32), wkv_b and scale.  Row b*seqlen + s is the query at position s of
+    sequence b: end_pos = s + 1 (causal), and its index row holds
+    min(K, s + 1) distinct positions of [0, s] in shuffled order (all of them
+    while s < K, as an indexer whose scores are causally masked returns),
+    -1 padded."""
+    gen = torch.Generator().manual_seed(seed)
+    R = B * seqlen
+    pos = torch.arange(R, dtype=torch.int64) % seqlen
+    topk = torch.full((R, K), -1, dtype=torch.int32)
+    for r in range(R):
+        s = int(pos[r])
+        n = min(K, s + 1)
+        sel = torch.randperm(s + 1, generator=gen)[:n]
+        topk[r, :n] = sel.to(torch.int32)
+    return {
+        "q_nope": _bf16_normal((R, H, D_NOPE), gen),
+        "q_pe": _bf16_normal((R, H, D_ROPE), gen),
+        "kv_cache": _bf16_normal((B, seqlen, D_LAT), gen),
+        "pe_cache": _bf16_normal((B, seqlen, D_ROPE), gen),
+        "cache_slot": (torch.arange(R, dtype=torch.int64) // seqlen).to(torch.int32),
+        "end_pos": (pos + 1).to(torch.int32),
+        "topk_idx": topk,
+        "wkv_b": _bf16_normal((H * (D_NOPE + D_V), D_LAT), gen, std=D_LAT ** -0.5),
+        "scale": SCALE,
+        "B": B, "seqlen": seqlen,
+    }

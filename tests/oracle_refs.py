@@ -13,6 +13,10 @@ a disagreement:
   output replaced by the given index row and the -inf/scatter mask built
   literally over all end_pos positions.
 
+* ``prefill_transcript``: the "MHA prefill" excerpt of the page "Queries"
+  (model.py 574-589) run as written in torch float64: every latent of the
+  chunk up-projected through wkv_b, keys joined with the shared rotary key,
+  the indexer's selection scattered into a -inf mask, the causal mask added.
 * ``transcript_projection``: the output projection of the page "Attention
   update" (model.py 607-608), ``self.wo(x.flatten(2))``, as torch's
   ``F.linear`` in float64 on the [B, 1, H, Dv] head outputs.
@@ -100,3 +104,25 @@ def transcript_projection(x, wo):
     x4 = xt.reshape(B, 1, -1, xt.shape[-1]) if xt.dim() == 3 else xt.reshape(B, 1, 1, -1)
     w = torch.as_tensor(to_f64(wo))
     return torch.nn.functional.linear(x4.flatten(2), w)[:, 0].numpy()
+
+
+def prefill_transcript(q_nope, q_pe, kv, k_pe, wkv_b, topk_indices, scale, Dv):
+    """q_nope [b,s,H,Dn], q_pe [b,s,H,Dr], kv [b,s,Dl] (the chunk's latents),
+    k_pe [b,s,Dr], wkv_b [H*(Dn+Dv), Dl], topk_indices [b,s,K] (positions in
+    [0, seqlen); ones after the query are removed by the causal mask).
+    Returns x [b,s,H,Dv]."""
+    qn, qp, kvt, kpe, wb = (torch.as_tensor(to_f64(a)) for a in (q_nope, q_pe, kv, k_pe, wkv_b))
+    bsz, seqlen, n_heads, qk_nope = qn.shape
+    q = torch.cat([qn, qp], dim=-1)
+    kvu = torch.nn.functional.linear(kvt, wb)
+    kvu = kvu.view(bsz, seqlen, n_heads, qk_nope + Dv)
+    k_nope, v = torch.split(kvu, [qk_nope, Dv], dim=-1)
+    k = torch.cat([k_nope, kpe.unsqueeze(2).expand(-1, -1, n_heads, -1)], dim=-1)
+    scores = torch.einsum("bshd,bthd->bsht", q, k).mul_(scale)
+    mask = torch.full((seqlen, seqlen), float("-inf"), dtype=torch.float64).triu_(1)
+    idx = torch.as_tensor(np.asarray(topk_indices), dtype=torch.int64)
+    index_mask = torch.full((bsz, seqlen, seqlen), float("-inf"), dtype=torch.float64).scatter_(-1, idx, 0)
+    index_mask += mask
+    scores += index_mask.unsqueeze(2)
+    scores = scores.softmax(dim=-1)
+    return torch.einsum("bsht,bthd->bshd", scores, v).numpy()

@@ -178,3 +178,19 @@ def test_projection_rejects_bad_arguments_without_a_launch(lib):
     assert call_p(dim=100) == INVALID_ARG
     assert call_p(K=0) == INVALID_ARG
     assert call_p(scale=float("nan")) == INVALID_ARG
+
+
+def test_prefill_rejects_bad_arguments_without_a_launch(lib):
+    A = 0x10000
+    args = [_fake(A)] * 4
+
+    def call(slot=_fake(A), n_slots=2, R=4, K=16, S=32, scale=0.07):
+        return lib.mla_sparse_prefill(*args, slot, _fake(A), _fake(A), _fake(A), ctypes.c_float(scale), _fake(A), R,
+                                      K, S, n_slots, _fake(A), 1 << 30, None, None, None)
+
+    assert call(slot=None) == INVALID_ARG
+    assert call(slot=_fake(A + 4)) == INVALID_ARG
+    assert call(n_slots=0) == INVALID_ARG
+    assert call(R=0) == INVALID_ARG
+    assert call(K=0) == INVALID_ARG
+    assert call(scale=float("inf")) == INVALID_ARG

@@ -12,6 +12,9 @@ the pages and the mathematics fix:
       excerpt's einsums run literally in torch float64;
   plus closed forms (one selected key; zero query) and set semantics of the
   index list (order, duplicates, padding).
+The per-row cache slot (one row per query position of a sequence) is pinned
+by the page's "MHA prefill" excerpt (page "Queries") run as written in torch
+float64 with the causal and index masks.
 The output projection (page "Attention update") is pinned by a hand-derived
 case, basis vectors (a unit input picks one column of wo), linearity, BLAS
 float64 matmul, and the page's ``wo(x.flatten(2))`` in torch float64.
@@ -26,7 +29,8 @@ import pytest
 import torch
 
 import oracle
-from tests.oracle_refs import nonabsorbed, transcript, transcript_projection, to_f64, valid_set
+from tests.oracle_refs import (nonabsorbed, prefill_transcript, transcript, transcript_projection, to_f64,
+                               valid_set)
 from sparse_latent_attention_absorb_b200 import workloads as wl
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -392,3 +396,60 @@ def test_projection_row_subset_matches_full_run():
     np.testing.assert_array_equal(part, full[[4, 0]])
     with pytest.raises(RuntimeError):
         oracle.output_projection(d["x"], d["wo"], rows=[5])
+
+
+# ---------------------------------------------------------------- prefill rows (page "Queries")
+
+def _prefill_case(rng, bsz, seqlen, K, H, Dn, Dr, Dl, Dv):
+    q_nope = rng.standard_normal((bsz, seqlen, H, Dn))
+    q_pe = rng.standard_normal((bsz, seqlen, H, Dr))
+    kv = rng.standard_normal((bsz, seqlen, Dl))
+    k_pe = rng.standard_normal((bsz, seqlen, Dr))
+    wkv_b = rng.standard_normal((H * (Dn + Dv), Dl)) / math.sqrt(Dl)
+    # the indexer returns K positions of the chunk for every query; with its
+    # scores causally masked the query's own position is among them, later
+    # ones may follow (the causal mask removes them)
+    topk = np.zeros((bsz, seqlen, K), np.int64)
+    for b in range(bsz):
+        for s_ in range(seqlen):
+            others = [t for t in rng.permutation(seqlen) if t != s_][:K - 1]
+            topk[b, s_] = [s_] + others
+    return q_nope, q_pe, kv, k_pe, wkv_b, topk.astype(np.int32)
+
+
+def _prefill_oracle(q_nope, q_pe, kv, k_pe, wkv_b, topk, scale, **kw):
+    bsz, seqlen, H = q_nope.shape[:3]
+    R = bsz * seqlen
+    slot = np.repeat(np.arange(bsz, dtype=np.int32), seqlen)
+    end_pos = np.tile(np.arange(1, seqlen + 1, dtype=np.int32), bsz)
+    return oracle.mla_sparse_decode(q_nope.reshape(R, H, -1), q_pe.reshape(R, H, -1), kv, k_pe, end_pos,
+                                    topk.reshape(R, -1), wkv_b, scale, cache_slot=slot, **kw)
+
+
+@pytest.mark.parametrize("dims", [dict(H=2, Dn=4, Dr=2, Dl=6, Dv=3, bsz=2, seqlen=7, K=3),
+                                  dict(H=128, Dn=128, Dr=64, Dl=512, Dv=128, bsz=1, seqlen=10, K=4)])
+def test_prefill_rows_equal_page_prefill_excerpt(dims):
+    rng = np.random.default_rng(21)
+    d = dict(dims)
+    bsz, seqlen, K = d.pop("bsz"), d.pop("seqlen"), d.pop("K")
+    case = _prefill_case(rng, bsz, seqlen, K, **d)
+    scale = (d["Dn"] + d["Dr"]) ** -0.5
+    got = _prefill_oracle(*case, scale).out.reshape(bsz, seqlen, d["H"], d["Dv"])
+    ref = prefill_transcript(*case, scale, d["Dv"])
+    assert rel_err(got, ref) < 1e-10
+
+
+def test_prefill_slot_out_of_range_gives_an_empty_row():
+    rng = np.random.default_rng(22)
+    q_nope, q_pe, kv, k_pe, wkv_b, topk = _prefill_case(rng, 2, 5, 3, H=2, Dn=4, Dr=2, Dl=6, Dv=3)
+    R = 10
+    slot = np.repeat(np.arange(2, dtype=np.int32), 5)
+    slot[3], slot[7] = 2, -1
+    end_pos = np.tile(np.arange(1, 6, dtype=np.int32), 2)
+    res = oracle.mla_sparse_decode(q_nope.reshape(R, 2, 4), q_pe.reshape(R, 2, 2), kv, k_pe, end_pos,
+                                   topk.reshape(R, 3), wkv_b, 0.4, cache_slot=slot)
+    for r in (3, 7):
+        assert np.all(res.out[r] == 0.0) and np.all(res.lse[r] == -np.inf)
+    good = [r for r in range(R) if r not in (3, 7)]
+    ref = _prefill_oracle(q_nope, q_pe, kv, k_pe, wkv_b, topk, 0.4)
+    np.testing.assert_array_equal(res.out[good], ref.out[good])

@@ -390,3 +390,57 @@ def test_decode_project_matches_oracle_chain(name):
     got = delta.double().cpu().numpy()
     assert got.shape == (B, wl.D_MODEL)
     assert np.max(np.abs(got - ref)) <= out_bound(ref)
+
+
+# ------------------------------------------------------------------ sparse prefill (page "Queries", prefill mode)
+
+def _prefill_dev(d):
+    return {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+@pytest.mark.parametrize("B,seqlen,K", [(2, 300, 128), (1, 700, 256)])
+def test_prefill_matches_oracle(B, seqlen, K):
+    """One row per query position, each reading its sequence's latents up to
+    its causal bound (rows with fewer than K valid positions included)."""
+    d = wl.generate_prefill(B, seqlen, K, seed=2200 + seqlen)
+    g = _prefill_dev(d)
+    R = B * seqlen
+    lse = torch.full((R, 128), float("nan"), dtype=torch.float32, device=DEV)
+    out = pkg.mla_sparse_prefill(g["q_nope"], g["q_pe"], g["kv_cache"], g["pe_cache"], g["cache_slot"], g["end_pos"],
+                                 g["topk_idx"], g["wkv_b"], g["scale"], lse_out=lse)
+    torch.cuda.synchronize()
+    rows = sorted({0, 1, 2, K - 2, K - 1, K, K + 1, seqlen - 1, seqlen, R // 2, R - 1} & set(range(R)))
+    ref = oracle.mla_sparse_decode(d["q_nope"], d["q_pe"], d["kv_cache"], d["pe_cache"], d["end_pos"],
+                                   d["topk_idx"], d["wkv_b"], d["scale"], rows=rows, cache_slot=d["cache_slot"])
+    got = out.double().cpu().numpy()[rows]
+    assert np.max(np.abs(got - ref.out)) <= out_bound(ref.out)
+    assert np.max(np.abs(lse.double().cpu().numpy()[rows] - ref.lse)) <= 1e-2
+
+
+def test_prefill_with_identity_slots_equals_decode():
+    d = wl.generate("small_b5_ctx40-700_top333")
+    g = to_dev(d)
+    B = d["q_nope"].shape[0]
+    slots = torch.arange(B, dtype=torch.int32, device=DEV)
+    out_p = pkg.mla_sparse_prefill(g["q_nope"], g["q_pe"], g["kv_cache"], g["pe_cache"], slots, g["end_pos"],
+                                   g["topk_idx"], g["wkv_b"], g["scale"])
+    out_d, _ = gpu_decode(g, lse=False)
+    assert torch.equal(out_p, out_d)
+
+
+def test_prefill_rows_with_an_out_of_range_slot_are_empty():
+    d = wl.generate_prefill(2, 70, 32, seed=2300)
+    g = _prefill_dev(d)
+    R = 140
+    lse = torch.empty((R, 128), dtype=torch.float32, device=DEV)
+    good = pkg.mla_sparse_prefill(g["q_nope"], g["q_pe"], g["kv_cache"], g["pe_cache"], g["cache_slot"], g["end_pos"],
+                                  g["topk_idx"], g["wkv_b"], g["scale"]).clone()
+    slots = g["cache_slot"].clone()
+    slots[5], slots[100] = 2, -7
+    out = pkg.mla_sparse_prefill(g["q_nope"], g["q_pe"], g["kv_cache"], g["pe_cache"], slots, g["end_pos"],
+                                 g["topk_idx"], g["wkv_b"], g["scale"], lse_out=lse)
+    torch.cuda.synchronize()
+    for r in (5, 100):
+        assert torch.all(out[r] == 0) and torch.all(torch.isneginf(lse[r]))
+    keep = [r for r in range(R) if r not in (5, 100)]
+    assert torch.equal(out[keep], good[keep])
