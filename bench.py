@@ -77,6 +77,24 @@ def source_hash():
     return h.hexdigest()[:16]
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank contributes its own device-timed
+    milliseconds, all of them get the maximum (a no-op with one rank).  Every
+    rank must call it at the same point (it is a collective)."""
+    if world <= 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(rows_per_rank: int, world: int, steps: int, ms: float) -> float:
+    """Queries per second of the whole job: every rank decodes its own batch
+    of rows_per_rank rows per step (weak scaling, replicas), timed by the
+    slowest rank."""
+    return rows_per_rank * world * steps / (ms / 1e3)
+
+
 def ncu_traffic(workload):
     """DRAM bytes per launch of the sparse-attend kernel from the committed ncu
     summary, if it was taken on the current kernel source."""
@@ -295,13 +313,9 @@ def gpu_arm(args, rank, world, device):
         clocks.mark_end()
     barrier()
     torch.cuda.synchronize()
-    elapsed_ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), world, device)
     ms_per_step = elapsed_ms / args.steps
-    value = B * world * args.steps / (elapsed_ms / 1e3)
+    value = whole_job_rate(B, world, args.steps, elapsed_ms)
     launches = 3 * args.steps
 
     # ---- per-kernel live timing (same stream, back-to-back launches, sets rotate)
@@ -432,11 +446,8 @@ def gpu_arm(args, rank, world, device):
         torch.cuda.synchronize()
         e_ms = f0.elapsed_time(f1)
         print(f"e2e: {args.steps} steps, host enqueue {host_ms:.1f} ms, device {e_ms:.1f} ms", file=sys.stderr)
-        if world > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=device)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": B * world * args.steps / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e_ms = max_over_ranks(e_ms, world, device)
+        e2e = {"value": whole_job_rate(B, world, args.steps, e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
                "how": "per step one mla_sparse_decode_host call (pinned host inputs uploaded, decode, result read "
                       "back on the call's stream); steps alternate between two streams"}
