@@ -143,6 +143,21 @@ int encode_wo(CUtensorMap* m, const void* wo, int dim) {
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// wo viewed as a 4-D bf16 tensor (64 k, 8 rows of a group, 256 k-blocks,
+// dim/8 groups) with strides (2 B, 32 KB, 128 B, 256 KB): one box {64, 8, 4, 16}
+// is 128 rows x 4 consecutive k-blocks, each row's four 128-byte pieces read
+// back to back, landing as [group][k-block][row][128 B] (128-byte swizzle).
+int encode_wo4(CUtensorMap* m, const void* wo, int dim) {
+  cuuint64_t dims[4] = {(cuuint64_t)kProjKBlock, 8, (cuuint64_t)kProjKBlocks, (cuuint64_t)dim / 8};
+  cuuint64_t strides[3] = {(cuuint64_t)kProjK * 2, (cuuint64_t)kProjKBlock * 2, (cuuint64_t)kProjK * 2 * 8};
+  cuuint32_t box[4] = {(cuuint32_t)kProjKBlock, 8, (cuuint32_t)kProjKGroupWide, (cuuint32_t)(kProjM / 8)};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(wo), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
 // The projection input x as a 2-D bf16 tensor [B rows, 16384 columns], boxes
 // of 64 columns x n_tile rows, 128-byte swizzle (rows past B read as zero).
 int encode_proj_x(CUtensorMap* m, const void* x, int B, int n_tile) {
@@ -189,7 +204,7 @@ bool proj_sizes_ok(int B, int dim) {
 // (f32 partials, then the reduce kernel), otherwise one CTA per tile writes
 // bf16 directly.
 struct ProjPlan {
-  int n_tile = 0, tiles = 0, n_ctas = 0;
+  int n_tile = 0, tiles = 0, n_ctas = 0, kgroup = 1;
   bool direct = false;
   size_t partial_bytes = 0;
 };
@@ -200,7 +215,14 @@ ProjPlan plan_projection(int B, int dim, int sm_count) {
   p.n_tile = ceil_div(ceil_div(B, y_tiles), 16) * 16;
   p.tiles = y_tiles * (dim / kProjM);
   p.direct = p.tiles >= sm_count;
-  p.n_ctas = p.direct ? p.tiles : sm_count;  // fewer CTAs than tiles x 256 units: a range spans <= 2 tiles
+  // four k-blocks per unit where two such stages fit (split mode only: a
+  // direct CTA's tile is 256 units of one k-block)
+  p.kgroup = (!p.direct && p.n_tile <= kProjWideNMax) ? kProjKGroupWide : 1;
+  // split mode: at most one CTA per unit (every CTA owns at least one unit, so
+  // the reduce's contributors are exactly the CTAs between a tile's first and
+  // last unit) and more CTAs than tiles (a range spans at most two tiles)
+  const long long units = (long long)p.tiles * (kProjKBlocks / p.kgroup);
+  p.n_ctas = p.direct ? p.tiles : (int)(units < sm_count ? units : sm_count);
   p.partial_bytes = p.direct ? 0 : (size_t)2 * p.n_ctas * p.n_tile * kProjM * sizeof(float);
   return p;
 }
@@ -294,19 +316,24 @@ int launch_combine(const void* o_part, const float* lse_part, const void* wkv_b,
 // it requests its first weight stages before waiting for that kernel.
 int launch_projection(const void* x, const void* wo, void* delta, int B, int dim, const ProjPlan& p, void* partial,
                       int* d_status, cudaStream_t stream, bool pdl) {
-  CUtensorMap tm_wo, tm_x;
+  CUtensorMap tm_wo, tm_wo4, tm_x;
   int rc;
   if ((rc = encode_wo(&tm_wo, wo, dim)) != MLA_OK) return rc;
+  if (p.kgroup == 1)
+    tm_wo4 = tm_wo;  // unused
+  else if ((rc = encode_wo4(&tm_wo4, wo, dim)) != MLA_OK)
+    return rc;
   if ((rc = encode_proj_x(&tm_x, x, B, p.n_tile)) != MLA_OK) return rc;
-  if ((rc = launch_ex(projection_kernel, dim3((unsigned)p.n_ctas), dim3(kProjThreads), proj_smem_bytes(p.n_tile),
-                      stream, pdl, tm_wo, tm_x, static_cast<float*>(partial), static_cast<__nv_bfloat16*>(delta), B,
-                      dim, p.n_tile, p.n_ctas, p.direct ? 1 : 0, d_status)) != MLA_OK)
+  if ((rc = launch_ex(projection_kernel, dim3((unsigned)p.n_ctas), dim3(kProjThreads),
+                      proj_smem_bytes(p.n_tile, p.kgroup), stream, pdl, tm_wo, tm_wo4, tm_x,
+                      static_cast<float*>(partial), static_cast<__nv_bfloat16*>(delta), B, dim, p.n_tile, p.n_ctas,
+                      p.direct ? 1 : 0, p.kgroup, d_status)) != MLA_OK)
     return rc;
   if (p.direct) return MLA_OK;
   dim3 grid((unsigned)p.tiles, ceil_div(p.n_tile, kProjReduceRows));
   return launch_ex(projection_reduce_kernel, grid, dim3(kProjReduceThreads), 0, stream, true,
-                   static_cast<const float*>(partial),
-                   static_cast<__nv_bfloat16*>(delta), B, dim, p.n_tile, p.n_ctas);
+                   static_cast<const float*>(partial), static_cast<__nv_bfloat16*>(delta), B, dim, p.n_tile,
+                   p.n_ctas, p.kgroup);
 }
 
 int prepare(DeviceInfo** info) {

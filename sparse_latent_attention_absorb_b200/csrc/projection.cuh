@@ -46,23 +46,34 @@ constexpr int kProjABytes = kProjM * kProjKBlock * 2;  // 16 KB
 constexpr int kProjThreads = 192;
 constexpr int kProjReduceRows = 16;                // batch rows per reduce CTA
 
-__host__ __device__ constexpr int proj_stage_bytes(int n_tile) { return kProjABytes + n_tile * kProjKBlock * 2; }
-__host__ __device__ constexpr int proj_stages(int n_tile) {
-  return kProjStageBudget / proj_stage_bytes(n_tile) < kProjStagesMax ? kProjStageBudget / proj_stage_bytes(n_tile)
-                                                                      : kProjStagesMax;
+// A unit covers kgroup consecutive k-blocks: 1, or kProjKGroupWide when the
+// batch tile is narrow enough for two such stages (then the wo box reads four
+// consecutive 128-byte pieces of every row back to back).
+constexpr int kProjKGroupWide = 4;
+constexpr int kProjWideNMax = 64;  // widest batch tile that uses kProjKGroupWide
+__host__ __device__ constexpr int proj_stage_bytes(int n_tile, int kgroup) {
+  return kgroup * (kProjABytes + n_tile * kProjKBlock * 2);
+}
+__host__ __device__ constexpr int proj_stages(int n_tile, int kgroup) {
+  return kProjStageBudget / proj_stage_bytes(n_tile, kgroup) < kProjStagesMax
+             ? kProjStageBudget / proj_stage_bytes(n_tile, kgroup)
+             : kProjStagesMax;
 }
 // shared memory of one CTA: the ring, barriers, alignment pad
-__host__ __device__ constexpr int proj_smem_bytes(int n_tile) {
-  return proj_stages(n_tile) * proj_stage_bytes(n_tile) + 256 + kSmemAlignPad;
+__host__ __device__ constexpr int proj_smem_bytes(int n_tile, int kgroup) {
+  return proj_stages(n_tile, kgroup) * proj_stage_bytes(n_tile, kgroup) + 256 + kSmemAlignPad;
 }
-// the largest of them, over the batch tiles the host can choose
+// the largest of them, over the batch tiles and unit widths the host can choose
 constexpr int proj_smem_max() {
   int m = 0;
-  for (int n = 16; n <= kProjNMax; n += 16) m = proj_smem_bytes(n) > m ? proj_smem_bytes(n) : m;
+  for (int n = 16; n <= kProjNMax; n += 16) {
+    m = proj_smem_bytes(n, 1) > m ? proj_smem_bytes(n, 1) : m;
+    if (n <= kProjWideNMax) m = proj_smem_bytes(n, kProjKGroupWide) > m ? proj_smem_bytes(n, kProjKGroupWide) : m;
+  }
   return m;
 }
 static_assert(proj_smem_max() <= 232448, "shared memory");
-static_assert(proj_stages(kProjNMax) >= 2, "ring depth");
+static_assert(proj_stages(kProjNMax, 1) >= 2 && proj_stages(kProjWideNMax, kProjKGroupWide) >= 2, "ring depth");
 
 // First unit of CTA c when U units are spread over C CTAs.
 __host__ __device__ __forceinline__ long long proj_unit_begin(long long c, long long U, long long C) {
@@ -75,24 +86,42 @@ __host__ __device__ __forceinline__ int proj_cta_of_unit(long long x, long long 
 }
 
 __global__ void __launch_bounds__(kProjThreads, 1)
-projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_x,
-                  float* __restrict__ partial, __nv_bfloat16* __restrict__ delta, int B, int dim, int n_tile,
-                  int n_ctas, int direct, int* d_status) {
+projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_wo4,
+                  const __grid_constant__ CUtensorMap tm_x, float* __restrict__ partial,
+                  __nv_bfloat16* __restrict__ delta, int B, int dim, int n_tile, int n_ctas, int direct, int kgroup,
+                  int* d_status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
-  const int stages = proj_stages(n_tile);
-  const int stage_bytes = proj_stage_bytes(n_tile);
+  const int stages = proj_stages(n_tile, kgroup);
+  const int stage_bytes = proj_stage_bytes(n_tile, kgroup);
+  const int upt = kProjKBlocks / kgroup;        // units per tile
+  const int a_bytes = kgroup * kProjABytes;     // wo part of a stage; the x boxes follow
   const int m_tiles = dim / kProjM;
-  const long long U = (long long)m_tiles * ((B + n_tile - 1) / n_tile) * kProjKBlocks;
+  const long long U = (long long)m_tiles * ((B + n_tile - 1) / n_tile) * upt;
   const long long u0 = proj_unit_begin(c, U, n_ctas);
   const int n_units = (int)(proj_unit_begin(c + 1, U, n_ctas) - u0);
-  const long long t0 = u0 / kProjKBlocks;  // first tile of this CTA
-  const int n_seg = n_units > 0 ? (int)((u0 + n_units - 1) / kProjKBlocks - t0) + 1 : 0;  // <= 2
-  // unit u: tile u / 256 = y * m_tiles + m, k-block u % 256
-  auto unit_m = [&](long long u) { return (int)((u / kProjKBlocks) % m_tiles); };
-  auto unit_row0 = [&](long long u) { return (int)((u / kProjKBlocks) / m_tiles) * n_tile; };
+  const long long t0 = u0 / upt;  // first tile of this CTA
+  const int n_seg = n_units > 0 ? (int)((u0 + n_units - 1) / upt - t0) + 1 : 0;  // <= 2
+  // unit u: tile u / upt = y * m_tiles + m, first k-block (u % upt) * kgroup
+  auto unit_m = [&](long long u) { return (int)((u / upt) % m_tiles); };
+  auto unit_row0 = [&](long long u) { return (int)((u / upt) / m_tiles) * n_tile; };
+  auto unit_kb0 = [&](long long u) { return (int)(u % upt) * kgroup; };
+  // wo part of a unit: one 2-D box [128 rows x 64], or with kgroup = 4 one
+  // 4-D box over (64 k, 8 rows, 4 k-blocks, 16 row groups), which lands as
+  // [group][k-block][row][128 B]: 8-row x 128-byte swizzle atoms, the groups
+  // 4 KB apart, k-block j at j KB
+  auto load_wo = [&](uint32_t dst, uint32_t bar, long long u) {
+    if (kgroup == 1)
+      tma_load_2d(dst, &tm_wo, bar, unit_kb0(u) * kProjKBlock, unit_m(u) * kProjM);
+    else
+      tma_load_4d(dst, &tm_wo4, bar, 0, 0, unit_kb0(u), unit_m(u) * (kProjM / 8));
+  };
+  auto load_x = [&](uint32_t dst, uint32_t bar, long long u) {
+    for (int j = 0; j < kgroup; ++j)
+      tma_load_2d(dst + j * n_tile * kProjKBlock * 2, &tm_x, bar, (unit_kb0(u) + j) * kProjKBlock, unit_row0(u));
+  };
 
   const uint32_t sRing = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
@@ -130,31 +159,24 @@ projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_consta
   if (warp == 4) {
     // ------------------------------------------------------------ TMA
     if (lane == 0 && n_units > 0) {
-      tma_prefetch_desc(&tm_wo);
+      tma_prefetch_desc(kgroup == 1 ? &tm_wo : &tm_wo4);
       tma_prefetch_desc(&tm_x);
       // The first stages' weights go out before the wait on the kernel that
       // writes x (programmatic dependent launch): wo does not depend on it.
       const int pre = n_units < stages ? n_units : stages;
       for (int i = 0; i < pre; ++i) {
-        const long long u = u0 + i;
         mbar_arrive_expect_tx(full(i), stage_bytes);
-        tma_load_2d(sRing + i * stage_bytes, &tm_wo, full(i), (int)(u % kProjKBlocks) * kProjKBlock,
-                    unit_m(u) * kProjM);
+        load_wo(sRing + i * stage_bytes, full(i), u0 + i);
       }
       grid_dep_wait();
-      for (int i = 0; i < pre; ++i) {
-        const long long u = u0 + i;
-        tma_load_2d(sRing + i * stage_bytes + kProjABytes, &tm_x, full(i), (int)(u % kProjKBlocks) * kProjKBlock,
-                    unit_row0(u));
-      }
+      for (int i = 0; i < pre; ++i) load_x(sRing + i * stage_bytes + a_bytes, full(i), u0 + i);
       for (int i = pre, st = pre % stages; i < n_units; ++i, st = (st + 1 == stages) ? 0 : st + 1) {
         const long long u = u0 + i;
         wait(empty(st), ((i / stages) - 1) & 1, ab);
         const uint32_t dst = sRing + st * stage_bytes;
         mbar_arrive_expect_tx(full(st), stage_bytes);
-        const int kx = (int)(u % kProjKBlocks) * kProjKBlock;
-        tma_load_2d(dst, &tm_wo, full(st), kx, unit_m(u) * kProjM);
-        tma_load_2d(dst + kProjABytes, &tm_x, full(st), kx, unit_row0(u));
+        load_wo(dst, full(st), u);
+        load_x(dst + a_bytes, full(st), u);
       }
     }
     __syncwarp();
@@ -165,19 +187,24 @@ projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_consta
       int seg = 0;
       for (int i = 0, st = 0; i < n_units; ++i, st = (st + 1 == stages) ? 0 : st + 1) {
         const long long u = u0 + i;
-        const bool first = (i == 0) || (u % kProjKBlocks == 0);
-        const bool last = (i == n_units - 1) || ((u + 1) % kProjKBlocks == 0);
+        const bool first = (i == 0) || (u % upt == 0);
+        const bool last = (i == n_units - 1) || ((u + 1) % upt == 0);
         const int acc = seg & 1;
         if (first && seg >= 2) wait(acc_empty(acc), ((seg - 2) >> 1) & 1, ab);
         wait(full(st), (i / stages) & 1, ab);
         tc_fence_after();
         const uint32_t a0 = sRing + st * stage_bytes;
-        const uint32_t b0 = a0 + kProjABytes;
+        const uint32_t b0 = a0 + a_bytes;
+        // wo k-block j: the 2-D box (8-row groups 1 KB apart), or block j of
+        // the 4-D box (groups 4 KB apart, block j at j KB)
+        const uint32_t a_sbo = kgroup == 1 ? 1024u : 4096u;
+        for (int j = 0; j < kgroup; ++j) {
 #pragma unroll
-        for (int k = 0; k < kProjKBlock / 16; ++k) {  // 32 bytes of k per step inside the 128-byte rows
-          const uint64_t a = smem_desc_sw128(a0 + k * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(b0 + k * 32, 16, 1024);
-          mma_ss(tmem + acc * acc_cols, a, bd, idesc, (first && k == 0) ? 0u : 1u);
+          for (int k = 0; k < kProjKBlock / 16; ++k) {  // 32 bytes of k per step inside the 128-byte rows
+            const uint64_t a = smem_desc_sw128(a0 + j * 1024 + k * 32, 16, a_sbo);
+            const uint64_t bd = smem_desc_sw128(b0 + j * n_tile * kProjKBlock * 2 + k * 32, 16, 1024);
+            mma_ss(tmem + acc * acc_cols, a, bd, idesc, (first && j == 0 && k == 0) ? 0u : 1u);
+          }
         }
         mma_commit(empty(st));
         if (last) {
@@ -196,7 +223,7 @@ projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_consta
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     for (int seg = 0; seg < n_seg; ++seg) {
       const int acc = seg & 1;
-      const long long u_seg = (t0 + seg) * kProjKBlocks;
+      const long long u_seg = (t0 + seg) * upt;
       const int row0 = unit_row0(u_seg);
       wait(acc_full(acc), (seg >> 1) & 1, ab);
       tc_fence_after();
@@ -239,23 +266,24 @@ constexpr int kProjReduceThreads = kProjReduceRows * 32;
 
 __global__ void __launch_bounds__(kProjReduceThreads)
 projection_reduce_kernel(const float* __restrict__ partial, __nv_bfloat16* __restrict__ delta, int B, int dim,
-                         int n_tile, int n_ctas) {
+                         int n_tile, int n_ctas, int kgroup) {
   const int t = blockIdx.x;
   const int m_tiles = dim / kProjM;
   const int m = t % m_tiles;
   const int row0 = (t / m_tiles) * n_tile;
   const int j = blockIdx.y * kProjReduceRows + (int)(threadIdx.x >> 5);  // row within the tile
   const int n4 = (int)(threadIdx.x & 31) * 4;
-  const int U = m_tiles * ((B + n_tile - 1) / n_tile) * kProjKBlocks;
-  const int first_unit = t * kProjKBlocks;
-  const int c_lo = ((first_unit + 1) * n_ctas - 1) / U;              // CTA holding the tile's first unit
-  const int c_hi = ((first_unit + kProjKBlocks) * n_ctas - 1) / U;   // ... and its last
+  const int upt = kProjKBlocks / kgroup;  // units per tile
+  const int U = m_tiles * ((B + n_tile - 1) / n_tile) * upt;
+  const int first_unit = t * upt;
+  const int c_lo = ((first_unit + 1) * n_ctas - 1) / U;     // CTA holding the tile's first unit
+  const int c_hi = ((first_unit + upt) * n_ctas - 1) / U;   // ... and its last
   grid_dep_wait();  // the partials come from projection_kernel
   if (j >= n_tile || row0 + j >= B) return;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
   for (int cc = c_lo; cc <= c_hi; ++cc) {
-    const int seg = (cc * U / n_ctas) / kProjKBlocks == t ? 0 : 1;  // the tile is cc's first or second segment
+    const int seg = (cc * U / n_ctas) / upt == t ? 0 : 1;  // the tile is cc's first or second segment
     const float4 v = __ldg(reinterpret_cast<const float4*>(partial + ((size_t)(2 * cc + seg) * n_tile + j) * kProjM + n4));
     acc.x += v.x;
     acc.y += v.y;

@@ -128,7 +128,10 @@ def test_projection_workspace_size_formula(lib):
         if tiles >= sms:
             assert got == 256  # one CTA per tile writes bf16 directly: no partials
         else:
-            assert got == 2 * sms * n_tile * 128 * 4  # two f32 partial slots per CTA
+            # units of four k-blocks for tiles of <= 64 rows, else of one; at
+            # most one CTA per unit; two f32 partial slots per CTA
+            units = tiles * (64 if n_tile <= 64 else 256)
+            assert got == 2 * min(sms, units) * n_tile * 128 * 4
     assert lib.mla_output_projection_workspace_size(1000, 7168) == 256  # 4 x 56 tiles >= 148 SMs
     for B, dim in ((0, 7168), (1, 0), (1, 100), (1, 7169), (1, 1 << 17)):
         assert lib.mla_output_projection_workspace_size(B, dim) == 0
