@@ -453,3 +453,39 @@ def test_prefill_slot_out_of_range_gives_an_empty_row():
     good = [r for r in range(R) if r not in (3, 7)]
     ref = _prefill_oracle(q_nope, q_pe, kv, k_pe, wkv_b, topk, 0.4)
     np.testing.assert_array_equal(res.out[good], ref.out[good])
+
+
+def test_next_rows_regression_fixture():
+    """Stored oracle outputs for per-row cache slots (prefill rows) and the
+    output projection (written by tests/golden/make_golden.py, which calls
+    only the oracle): guards against accidental changes of their arithmetic."""
+    with open(os.path.join(GOLDEN, "oracle_next_rows_regression.json")) as f:
+        g = json.load(f)
+    from tests.golden.make_golden import tiny_prefill_case, tiny_projection_case
+    p = tiny_prefill_case()
+    res = oracle.mla_sparse_decode(p["q_nope"], p["q_pe"], p["kv_cache"], p["pe_cache"], p["end_pos"],
+                                   p["topk_idx"], p["wkv_b"], p["scale"], cache_slot=p["cache_slot"])
+    np.testing.assert_allclose(res.out.reshape(-1), np.array(g["prefill_out"]), rtol=1e-13, atol=1e-15)
+    np.testing.assert_array_equal(np.isneginf(res.lse.reshape(-1)), np.isneginf(np.array(g["prefill_lse"])))
+    fin = np.isfinite(res.lse.reshape(-1))
+    np.testing.assert_allclose(res.lse.reshape(-1)[fin], np.array(g["prefill_lse"])[fin], rtol=1e-13)
+    j = tiny_projection_case()
+    np.testing.assert_allclose(oracle.output_projection(j["x"], j["wo"]).reshape(-1), np.array(g["projection"]),
+                               rtol=1e-13, atol=1e-15)
+
+
+def test_prefill_generator_structure():
+    """One row per query position: slot = its sequence, end_pos = position
+    + 1, and min(K, position + 1) distinct causally valid indices, -1 padded."""
+    d = wl.generate_prefill(2, 40, 16, seed=7)
+    R = 80
+    pos = np.arange(R) % 40
+    np.testing.assert_array_equal(d["cache_slot"].numpy(), np.arange(R) // 40)
+    np.testing.assert_array_equal(d["end_pos"].numpy(), pos + 1)
+    ti = d["topk_idx"].numpy()
+    for r in range(R):
+        n = min(16, pos[r] + 1)
+        sel = ti[r, :n]
+        assert len(set(sel.tolist())) == n and sel.min() >= 0 and sel.max() <= pos[r]
+        assert np.all(ti[r, n:] == -1)
+    assert tuple(d["kv_cache"].shape) == (2, 40, 512) and tuple(d["q_nope"].shape) == (R, 128, 128)
