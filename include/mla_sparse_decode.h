@@ -1,6 +1,11 @@
 /*
  * mla_sparse_decode.h -- C ABI of the B200 (sm_100a) sparse MLA decode library.
  *
+ * Also declared here, after the decode step: the sparse prefill over the same
+ * kernels (mla_sparse_prefill, page "Queries") and the attention output
+ * projection (mla_output_projection, mla_sparse_decode_project, page
+ * "Attention update").
+ *
  * One decode step of DeepSeek-V3.2-Exp's absorbed multi-head latent attention
  * with the indexer's top-k mask, as the atlas pages of
  * deepseek-ai/DeepSeek-V3.2-Exp inference/model.py (rev 87e509a2e5a1) show it:
@@ -35,7 +40,8 @@
  *     (the indexer's top-k output is); a repeated index would be counted twice.
  *     Index order is irrelevant.  A row with no valid index yields out = 0 and
  *     lse = -inf.
- *   - Batch row b reads cache slot b (the excerpt slices kv_cache[:bsz]).
+ *   - Batch row b reads cache slot b (the excerpt slices kv_cache[:bsz]);
+ *     mla_sparse_prefill gives each row its slot explicitly.
  */
 #ifndef MLA_SPARSE_DECODE_H
 #define MLA_SPARSE_DECODE_H
