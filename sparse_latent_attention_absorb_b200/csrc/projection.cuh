@@ -32,6 +32,7 @@
 #pragma once
 
 #include "kernels.cuh"
+#include "projection_plan.h"
 
 namespace mla {
 
@@ -75,16 +76,6 @@ constexpr int proj_smem_max() {
 static_assert(proj_smem_max() <= 232448, "shared memory");
 static_assert(proj_stages(kProjNMax, 1) >= 2 && proj_stages(kProjWideNMax, kProjKGroupWide) >= 2, "ring depth");
 
-// First unit of CTA c when U units are spread over C CTAs.
-__host__ __device__ __forceinline__ long long proj_unit_begin(long long c, long long U, long long C) {
-  return c * U / C;
-}
-// The CTA whose unit range contains unit x: the largest c with
-// proj_unit_begin(c) <= x, i.e. ceil((x + 1) C / U) - 1.
-__host__ __device__ __forceinline__ int proj_cta_of_unit(long long x, long long U, long long C) {
-  return (int)(((x + 1) * C - 1) / U);
-}
-
 __global__ void __launch_bounds__(kProjThreads, 1)
 projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_wo4,
                   const __grid_constant__ CUtensorMap tm_x, float* __restrict__ partial,
@@ -100,8 +91,8 @@ projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_consta
   const int a_bytes = kgroup * kProjABytes;     // wo part of a stage; the x boxes follow
   const int m_tiles = dim / kProjM;
   const long long U = (long long)m_tiles * ((B + n_tile - 1) / n_tile) * upt;
-  const long long u0 = proj_unit_begin(c, U, n_ctas);
-  const int n_units = (int)(proj_unit_begin(c + 1, U, n_ctas) - u0);
+  const long long u0 = proj_unit_begin<long long>(c, U, n_ctas);
+  const int n_units = (int)(proj_unit_begin<long long>(c + 1, U, n_ctas) - u0);
   const long long t0 = u0 / upt;  // first tile of this CTA
   const int n_seg = n_units > 0 ? (int)((u0 + n_units - 1) / upt - t0) + 1 : 0;  // <= 2
   // unit u: tile u / upt = y * m_tiles + m, first k-block (u % upt) * kgroup
@@ -275,15 +266,14 @@ projection_reduce_kernel(const float* __restrict__ partial, __nv_bfloat16* __res
   const int n4 = (int)(threadIdx.x & 31) * 4;
   const int upt = kProjKBlocks / kgroup;  // units per tile
   const int U = m_tiles * ((B + n_tile - 1) / n_tile) * upt;
-  const int first_unit = t * upt;
-  const int c_lo = ((first_unit + 1) * n_ctas - 1) / U;     // CTA holding the tile's first unit
-  const int c_hi = ((first_unit + upt) * n_ctas - 1) / U;   // ... and its last
+  int c_lo, c_hi;  // the CTAs holding the tile's units
+  proj_tile_ctas<int>(t, upt, U, n_ctas, &c_lo, &c_hi);
   grid_dep_wait();  // the partials come from projection_kernel
   if (j >= n_tile || row0 + j >= B) return;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
   for (int cc = c_lo; cc <= c_hi; ++cc) {
-    const int seg = (cc * U / n_ctas) / upt == t ? 0 : 1;  // the tile is cc's first or second segment
+    const int seg = proj_segment_of<int>(cc, t, upt, U, n_ctas);  // the tile is cc's first or second segment
     const float4 v = __ldg(reinterpret_cast<const float4*>(partial + ((size_t)(2 * cc + seg) * n_tile + j) * kProjM + n4));
     acc.x += v.x;
     acc.y += v.y;
