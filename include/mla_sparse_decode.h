@@ -287,6 +287,19 @@ int mla_sparse_decode_project(const void* q_nope, const void* q_pe, const void* 
                               const void* wo, void* delta, int B, int K, int S_max, int dim, void* workspace,
                               size_t workspace_bytes, float* lse_out, int* d_status, cudaStream_t stream);
 
+/*
+ * Self-test of the bounded waits every kernel relies on (no counterpart on the
+ * pages): launches one CTA whose thread waits, through the kernels' own wait,
+ * on a barrier that nothing arrives on.  After the wait limit (2 s) it must
+ * write MLA_ERR_DEVICE_TIMEOUT to *d_status (left unchanged if already
+ * non-zero) and return; *d_result receives 4 when the wait gave up, set the
+ * abort flag and a second wait returned at once (bit 0 / bit 1 set = a wait
+ * wrongly reported completion).  d_status, d_result: device ints, 4-byte
+ * aligned.  Takes about 2 s on the stream; the context stays usable.
+ * Returns an mla_status (of the launch).
+ */
+int mla_selftest_wait_timeout(int* d_status, int* d_result, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,8 @@ EXPORTS = ("mla_status_string", "mla_num_splits", "mla_sparse_decode_workspace_s
            "mla_absorb_q", "mla_sparse_attend", "mla_combine_value_up", "mla_sparse_decode_noalloc",
            "mla_sparse_decode_host_workspace_size", "mla_sparse_decode_host",
            "mla_output_projection_workspace_size", "mla_output_projection",
-           "mla_sparse_decode_project_workspace_size", "mla_sparse_decode_project", "mla_sparse_prefill")
+           "mla_sparse_decode_project_workspace_size", "mla_sparse_decode_project", "mla_sparse_prefill",
+           "mla_selftest_wait_timeout")
 STATIC_SCRATCH_BYTES = 32 << 20  # MLA_STATIC_SCRATCH_BYTES
 
 _lib = None
@@ -77,6 +78,8 @@ def load_library():
     lib.mla_sparse_decode_project.argtypes = [p, p, p, p, p, p, p, f, p, p, i, i, i, i, p, sz, p, p, p]
     lib.mla_sparse_prefill.restype = i
     lib.mla_sparse_prefill.argtypes = [p, p, p, p, p, p, p, p, f, p, i, i, i, i, p, sz, p, p, p]
+    lib.mla_selftest_wait_timeout.restype = i
+    lib.mla_selftest_wait_timeout.argtypes = [p, p, p]
     _lib = lib
     return lib
 
@@ -398,3 +401,15 @@ def mla_sparse_prefill(q_nope, q_pe, kv_cache, pe_cache, cache_slot, end_pos, to
                                 _stream(stream))
     _raise(rc, "mla_sparse_prefill")
     return out
+
+
+def selftest_wait_timeout(stream=None):
+    """Runs the bounded-wait self-test (about 2 s); returns (status word,
+    result bits) as the library wrote them: (MLA_ERR_DEVICE_TIMEOUT, 4) when
+    healthy."""
+    lib = load_library()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    result = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    _raise(lib.mla_selftest_wait_timeout(_ptr(status), _ptr(result), _stream(stream)), "mla_selftest_wait_timeout")
+    torch.cuda.synchronize()
+    return int(status.item()), int(result.item())

@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libmla_sparse_decode.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
-SOURCES = [os.path.join(CSRC, "mla_sparse_decode.cu")]
+SOURCES = [os.path.join(CSRC, "mla_sparse_decode.cu"), os.path.join(CSRC, "selftest.cu")]
 DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("kernels.cuh", "ptx.cuh", "projection.cuh", "projection_plan.h")] + [
     os.path.join(INCLUDE, "mla_sparse_decode.h")]
 
