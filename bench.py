@@ -1,13 +1,23 @@
 """Benchmark of the sparse absorbed MLA decode step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+                    [--no-extras] [--sets S]
 
 One step = one call of the whole decode path (absorb, sparse attend, combine +
 value-up) over one batch of B rows.  The default workload is the B=64,
 32K-context, top-2048 configuration.  Inputs are synthetic (seeded), generated
-on the host in bf16 and kept resident in HBM; NSETS independent input sets
-(queries, index sets, end positions and a separate copy of wkv_b each) rotate
-between steps, so a step never finds the previous step's bytes in L2.
+on the host in bf16 and kept resident in HBM; independent input sets
+(queries, index sets, end positions and a separate copy of wkv_b each, and the
+caches too when they are small) rotate between steps, enough of them that one
+rotation moves more than twice the L2 size, so a step never finds the
+previous step's bytes in L2.
+
+The timed region is a window of exactly K steps, bracketed by a barrier and a
+synchronize; windows are repeated until they span at least 0.5 s and the
+median window gives the step time (with NVML clock samples from all of them).
+The same line carries per-kernel cold timings, every other configuration of
+the pages (``per_config``), the output projection, the sparse prefill and the
+end-to-end figure through the host-buffer entry point.
 
 Prints one JSON line (rank 0).  Under torchrun every rank runs its own batch
 (weak scaling, no collective on the path); the step time is the maximum over
@@ -225,21 +235,139 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- GPU arm
 
-def make_sets(w, device):
-    """NSETS input sets on the device: the caches are shared (model state),
-    everything else is drawn per set."""
+L2_BYTES = 126 * 2 ** 20  # B200 L2 (the footprint rule below keeps a rotation at > 2x this)
+
+
+def n_rotating_sets(w, floor=NSETS):
+    """Input sets to rotate so that one rotation touches more than twice the
+    L2 size: each set holds its own wkv_b copy, queries, indices and, when the
+    workload's caches are small enough to stay in L2, its own caches."""
+    per_set = 128 * 256 * 512 * 2 + w.B * 128 * 192 * 2 + 4 * w.B * w.K
+    if own_caches(w):
+        per_set += w.B * w.S_max * 1152
+    return max(floor, math.ceil(2 * L2_BYTES / per_set))
+
+
+def own_caches(w):
+    """Caches smaller than twice L2 are drawn per input set (else the gathered
+    rows of one step would still be in L2 at the next)."""
+    return w.B * w.S_max * 1152 < 2 * L2_BYTES
+
+
+def make_sets(w, device, n_sets):
+    """n_sets input sets on the device.  Large caches are shared (model
+    state); queries, indices, end positions and a wkv_b copy are drawn per
+    set, and small caches too."""
     base = wl.generate(w)
-    caches = {k: base[k].to(device) for k in ("kv_cache", "pe_cache")}
+    shared = None if own_caches(w) else {k: base[k].to(device) for k in ("kv_cache", "pe_cache")}
     sets = []
-    for i in range(NSETS):
-        d = base if i == 0 else wl.generate(w, seed_offset=i, caches=False)
-        s = {k: d[k].to(device) for k in ("q_nope", "q_pe", "end_pos", "topk_idx", "wkv_b")}
-        s.update(caches)
+    for i in range(n_sets):
+        d = base if i == 0 else wl.generate(w, seed_offset=i, caches=shared is None)
+        keys = ("q_nope", "q_pe", "end_pos", "topk_idx", "wkv_b") + (("kv_cache", "pe_cache") if shared is None else ())
+        s = {k: d[k].to(device) for k in keys}
+        if shared is not None:
+            s.update(shared)
         s["scale"] = d["scale"]
         s["sum_k"] = wl.selected_count(d["end_pos"], d["topk_idx"])
         s["host"] = d
         sets.append(s)
     return sets, base
+
+
+def call_roofline(B, K, sum_k, ms_per_call):
+    hbm, tf, _, kind = peaks()
+    call_bytes, call_flops = algorithmic(B, K, sum_k)
+    t_hbm = call_bytes / (hbm * 1e9)
+    t_tc = call_flops / (tf * 1e12)
+    roof_ms = max(t_hbm, t_tc) * 1e3
+    return {"alg_bytes": call_bytes, "alg_flops": call_flops, "t_hbm_ms": t_hbm * 1e3, "t_tensor_ms": t_tc * 1e3,
+            "roofline_ms": roof_ms, "frac": roof_ms / ms_per_call, "bound": "hbm" if t_hbm >= t_tc else "tensor",
+            "peaks": {"hbm_gbs": hbm, "bf16_tflops": tf, "source": kind}}
+
+
+class Decoder:
+    """One graph-captured decode call per input set, and one graph of all the
+    sets' calls back to back (a replay = len(sets) steps)."""
+
+    def __init__(self, lib, w, sets, device, stream):
+        import ctypes
+        self.lib, self.w, self.sets, self.stream = lib, w, sets, stream
+        self.ws = torch.empty(lib.mla_sparse_decode_workspace_size(w.B, w.K, w.S_max), dtype=torch.uint8,
+                              device=device)
+        self.outs = [torch.empty((w.B, 128, 128), dtype=torch.bfloat16, device=device) for _ in sets]
+        P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+
+        def call(i, st):
+            s = sets[i]
+            rc = lib.mla_sparse_decode(P(s["q_nope"]), P(s["q_pe"]), P(s["kv_cache"]), P(s["pe_cache"]),
+                                       P(s["end_pos"]), P(s["topk_idx"]), P(s["wkv_b"]), ctypes.c_float(s["scale"]),
+                                       P(self.outs[i]), w.B, w.K, w.S_max, P(self.ws), self.ws.numel(), None, None,
+                                       ctypes.c_void_p(st.cuda_stream))
+            if rc != 0:
+                raise RuntimeError(f"mla_sparse_decode: status {rc}")
+
+        with torch.cuda.stream(stream):
+            for i in range(len(sets)):
+                call(i, stream)
+        stream.synchronize()
+        self.graphs = []
+        for i in range(len(sets)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                call(i, torch.cuda.current_stream())
+            self.graphs.append(g)
+        self.chain = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.chain, stream=stream):
+            for i in range(len(sets)):
+                call(i, torch.cuda.current_stream())
+        torch.cuda.synchronize()
+
+    def run(self, n):
+        """n decode steps, input sets in rotation."""
+        n_sets = len(self.sets)
+        with torch.cuda.stream(self.stream):
+            for _ in range(n // n_sets):
+                self.chain.replay()
+            for i in range(n % n_sets):
+                self.graphs[i].replay()
+
+    def time_ms(self, n):
+        """Device time of n steps (CUDA events on the launching stream)."""
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        self.run(n)
+        e1.record(self.stream)
+        self.stream.synchronize()
+        return e0.elapsed_time(e1)
+
+    def release(self):
+        self.graphs.clear()
+        self.chain = None
+
+
+def per_config(lib, device, stream, min_s=0.1):
+    """Every workload of the pages' configurations (the dense pass included),
+    each timed from graphs of back-to-back decode calls with its own rotating
+    input sets, with its whole-call roofline."""
+    out = {}
+    for name, w in wl.WORKLOADS.items():
+        sets, _ = make_sets(w, device, n_rotating_sets(w))
+        dec = Decoder(lib, w, sets, device, stream)
+        dec.run(2 * len(sets))
+        n = len(sets)
+        t = dec.time_ms(n)
+        reps = max(1, math.ceil(min_s * 1e3 / max(t, 1e-3)))
+        ms = dec.time_ms(n * reps) / (n * reps)
+        sum_k = statistics.mean(s["sum_k"] for s in sets)
+        out[name] = {"B": w.B, "K": w.K, "S_max": w.S_max, "sum_k_mean": sum_k, "splits": lib.mla_num_splits(w.B, w.K),
+                     "ms_per_call": ms, "queries_per_s": w.B / (ms * 1e-3), "calls_timed": n * reps,
+                     "rotating_sets": n, "own_caches_per_set": own_caches(w),
+                     "call_roofline": call_roofline(w.B, w.K, sum_k, ms)}
+        dec.release()
+        del dec, sets
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
 
 
 def gpu_arm(args, rank, world, device):
@@ -250,106 +378,81 @@ def gpu_arm(args, rank, world, device):
 
     lib = pkg.load_library()
     w = wl.ALL_WORKLOADS[args.workload]
-    sets, base = make_sets(w, device)
+    sets, base = make_sets(w, device, args.sets or n_rotating_sets(w))
     B, K, S_max = w.B, w.K, w.S_max
     n_split = pkg.num_splits(B, K)
-    ws = torch.empty(pkg.workspace_size(B, K, S_max), dtype=torch.uint8, device=device)
-    outs = [torch.empty((B, 128, 128), dtype=torch.bfloat16, device=device) for _ in sets]
     stream = torch.cuda.Stream(device=device)
+    dec = Decoder(lib, w, sets, device, stream)
     P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
-
-    def call(i, st):
-        s = sets[i]
-        rc = lib.mla_sparse_decode(P(s["q_nope"]), P(s["q_pe"]), P(s["kv_cache"]), P(s["pe_cache"]), P(s["end_pos"]),
-                                   P(s["topk_idx"]), P(s["wkv_b"]), ctypes.c_float(s["scale"]), P(outs[i]), B, K,
-                                   S_max, P(ws), ws.numel(), None, None, ctypes.c_void_p(st.cuda_stream))
-        if rc != 0:
-            raise binding.MLAError(rc, "mla_sparse_decode")
-
-    # One CUDA graph per input set (a replay is exactly one decode call), and
-    # one graph of NSETS consecutive calls, one per set, so that steps timed
-    # back to back do not each pay a graph launch.
-    with torch.cuda.stream(stream):
-        for i in range(len(sets)):
-            call(i, stream)
-    stream.synchronize()
-    graphs = []
-    for i in range(len(sets)):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            call(i, torch.cuda.current_stream())
-        graphs.append(g)
-    chain = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(chain, stream=stream):
-        for i in range(len(sets)):
-            call(i, torch.cuda.current_stream())
-    torch.cuda.synchronize()
-
-    def run_steps(n):
-        """n decode steps, input sets in rotation (n // NSETS chain replays, then singles)."""
-        for _ in range(n // NSETS):
-            chain.replay()
-        for i in range(n % NSETS):
-            graphs[i].replay()
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
-    # ---- timed region: K decode steps
-    with torch.cuda.stream(stream):
-        run_steps(args.warmup)
+    # ---- timed region: windows of exactly K decode steps, each bracketed by
+    # a barrier and a synchronize, repeated until the windows span >= 0.5 s;
+    # the median window (max over ranks) gives the step time
+    dec.run(args.warmup)
     stream.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    probe = max_over_ranks(dec.time_ms(args.steps), world, device)
+    repeats = max(1, min(100000, math.ceil(500.0 / max(probe, 1e-3))))
+    windows = []
     with ClockSampler(torch.cuda.current_device() if device.index is None else device.index) as clocks:
-        with torch.cuda.stream(stream):
-            clocks.mark_start()
-            ev0.record(stream)
-            run_steps(args.steps)
-            ev1.record(stream)
-        stream.synchronize()
+        clocks.mark_start()
+        for _ in range(repeats):
+            barrier()
+            torch.cuda.synchronize()
+            windows.append(max_over_ranks(dec.time_ms(args.steps), world, device))
         clocks.mark_end()
     barrier()
     torch.cuda.synchronize()
-    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), world, device)
-    ms_per_step = elapsed_ms / args.steps
-    value = whole_job_rate(B, world, args.steps, elapsed_ms)
+    window_ms = statistics.median(windows)
+    ms_per_step = window_ms / args.steps
+    value = whole_job_rate(B, world, args.steps, window_ms)
     launches = 3 * args.steps
 
-    # ---- per-kernel live timing (same stream, back-to-back launches, sets rotate)
+    # ---- per-kernel live timing, cold: graphs of back-to-back launches of one
+    # kernel on the same stream, input sets rotating, and for the two kernels
+    # that read only half of wkv_b each, enough wkv_b copies that a rotation of
+    # the halves they read exceeds L2
     q_lat = [torch.empty((B, 128, 512), dtype=torch.bfloat16, device=device) for _ in sets]
     # the attention kernel's per-split output: f32 partials, or the bf16 mixed
     # latent when each row is a single split
     o_part = (torch.empty((B, 128, 512), dtype=torch.bfloat16, device=device) if n_split == 1 else
               torch.empty((B, n_split, 128, 512), dtype=torch.float32, device=device))
     lse_part = torch.empty((B, n_split, 128), dtype=torch.float32, device=device)
+    n_w = max(len(sets), math.ceil(2 * L2_BYTES / (128 * 128 * 512 * 2)))
+    w_copies = [sets[i]["wkv_b"] if i < len(sets) else torch.empty_like(sets[0]["wkv_b"]).copy_(sets[i % len(sets)]["wkv_b"])
+                for i in range(n_w)]
     sv = ctypes.c_void_p(stream.cuda_stream)
+    ns = len(sets)
 
-    def k_absorb(i):
-        return lib.mla_absorb_q(P(sets[i]["q_nope"]), P(sets[i]["wkv_b"]), P(q_lat[i]), B, sv)
+    def k_absorb(r):
+        return lib.mla_absorb_q(P(sets[r % ns]["q_nope"]), P(w_copies[r % n_w]), P(q_lat[r % ns]), B, sv)
 
-    def k_attend(i):
-        s = sets[i]
-        return lib.mla_sparse_attend(P(q_lat[i]), P(s["q_pe"]), P(s["kv_cache"]), P(s["pe_cache"]), P(s["end_pos"]),
-                                     P(s["topk_idx"]), ctypes.c_float(s["scale"]), P(o_part), P(lse_part), B, K,
-                                     S_max, n_split, None, sv)
+    def k_attend(r):
+        s = sets[r % ns]
+        return lib.mla_sparse_attend(P(q_lat[r % ns]), P(s["q_pe"]), P(s["kv_cache"]), P(s["pe_cache"]),
+                                     P(s["end_pos"]), P(s["topk_idx"]), ctypes.c_float(s["scale"]), P(o_part),
+                                     P(lse_part), B, K, S_max, n_split, None, sv)
 
-    def k_combine(i):
-        return lib.mla_combine_value_up(P(o_part), P(lse_part), P(sets[i]["wkv_b"]), P(outs[i]), None, B, n_split, sv)
+    def k_combine(r):
+        return lib.mla_combine_value_up(P(o_part), P(lse_part), P(w_copies[r % n_w]), P(dec.outs[r % ns]), None, B,
+                                        n_split, sv)
 
     def time_kernel(fn, reps):
-        """Device time of one launch: `reps` back-to-back launches (input sets
-        rotating) captured in a CUDA graph, so host launch cost is excluded."""
+        """Device time of one launch: `reps` back-to-back launches captured in
+        a CUDA graph (host launch cost excluded), the second replay timed."""
         with torch.cuda.stream(stream):
             for r in range(4):
-                assert fn(r % NSETS) == 0
+                assert fn(r) == 0
         stream.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for r in range(reps):
-                fn(r % NSETS)
+                fn(r)
         with torch.cuda.stream(stream):
             g.replay()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -361,13 +464,86 @@ def gpu_arm(args, rank, world, device):
         return e0.elapsed_time(e1) / reps
 
     with torch.cuda.stream(stream):
-        for i in range(NSETS):
+        for i in range(ns):
             k_absorb(i)
     stream.synchronize()
-    reps = min(200, max(20, args.steps))
+    reps = 4 * max(ns, n_w) * 4
     t_absorb = time_kernel(k_absorb, reps)
     t_attend = time_kernel(k_attend, reps)
     t_combine = time_kernel(k_combine, reps)
+    del w_copies
+
+    extras = {}
+    if not args.no_extras:
+        extras = extra_measurements(args, lib, dec, sets, w, device, stream, rank, world)
+
+    # ---- roofline of the dominant kernel and of the whole call
+    hbm, tf, tf_sus, kind = peaks()
+    sum_k = statistics.mean(s["sum_k"] for s in sets)
+    a_bytes = attend_bytes(B, K, sum_k)
+    achieved = a_bytes / (t_attend * 1e-3) / 1e9
+    traffic = ncu_traffic(args.workload)
+    cr = call_roofline(B, K, sum_k, ms_per_step)
+
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "B": B, "heads": 128, "S_max": S_max, "K": K,
+                   "end_pos": list(w.end_pos), "index": w.index, "sum_k_mean": sum_k, "splits": n_split,
+                   "parallelism": f"replicas x{world} (batch rows)",
+                   "l2": f"{ns} rotating input sets (queries, indices, wkv_b copy each"
+                         f"{', caches' if own_caches(w) else ''}); a rotation moves {ns * cr['alg_bytes'] / 1e6:.0f} MB "
+                         f"> 2 x 126 MB L2",
+                   "timing": (f"{repeats} windows of exactly {args.steps} steps, each bracketed by a barrier and a "
+                              f"synchronize; median window ({statistics.median(windows):.3f} ms, min "
+                              f"{min(windows):.3f}, max {max(windows):.3f}); windows span "
+                              f"{sum(windows) / 1e3:.2f} s; CUDA graphs of consecutive steps, CUDA events on the "
+                              f"launching stream"),
+                   "windows": repeats},
+        "roofline": {"bound": "hbm", "kernel": "sparse_attend_kernel", "achieved": achieved, "peak": hbm,
+                     "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
+                     "peak_source": f"{kind} hbm_gbs (burst copy)", "alg_bytes_per_launch": a_bytes,
+                     "ms_per_launch": t_attend},
+        "call_roofline": cr,
+        "kernels_ms": {"absorb": t_absorb, "sparse_attend": t_attend, "combine_value_up": t_combine,
+                       "how": f"cold: graphs of {reps} back-to-back launches of one kernel, input sets rotating, "
+                              f"{n_w} wkv_b copies rotating for absorb and value-up"},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    res.update(extras)
+    dec.release()
+    return res, base
+
+
+def extra_measurements(args, lib, dec, sets, w, device, stream, rank, world):
+    """The other configurations, the rows after the path (output projection,
+    sparse prefill) and the end-to-end figure through the host-buffer API."""
+    import ctypes
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    sv = ctypes.c_void_p(stream.cuda_stream)
+    hbm = peaks()[0]
+    B, K, S_max = w.B, w.K, w.S_max
+
+    def time_graph(fn, reps):
+        with torch.cuda.stream(stream):
+            for r in range(2):
+                assert fn(r) == 0
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for r in range(reps):
+                fn(r)
+        with torch.cuda.stream(stream):
+            g.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        del g
+        return e0.elapsed_time(e1) / reps
 
     # ---- the step after the path: the output projection of the decode
     # outputs (page "Attention update"), wo [7168, 16384] bf16 = 235 MB, more
@@ -377,10 +553,11 @@ def gpu_arm(args, rank, world, device):
     p_delta = torch.empty((B, p_dim), dtype=torch.bfloat16, device=device)
     p_ws = torch.empty(lib.mla_output_projection_workspace_size(B, p_dim), dtype=torch.uint8, device=device)
 
-    def k_project(i):
-        return lib.mla_output_projection(P(outs[i]), P(p_wo), P(p_delta), B, p_dim, P(p_ws), p_ws.numel(), None, sv)
+    def k_project(r):
+        return lib.mla_output_projection(P(dec.outs[r % len(sets)]), P(p_wo), P(p_delta), B, p_dim, P(p_ws),
+                                         p_ws.numel(), None, sv)
 
-    t_project = time_kernel(k_project, min(50, reps))
+    t_project = time_graph(k_project, 50)
     p_bytes = p_dim * 16384 * 2 + B * 16384 * 2 + B * p_dim * 2
     del p_wo
 
@@ -394,110 +571,89 @@ def gpu_arm(args, rank, world, device):
     pf_out = torch.empty((R_pf, 128, 128), dtype=torch.bfloat16, device=device)
     pf_ws = torch.empty(lib.mla_sparse_decode_workspace_size(R_pf, K_pf, S_pf), dtype=torch.uint8, device=device)
 
-    def k_prefill(i):
+    def k_prefill(r):
         return lib.mla_sparse_prefill(P(pfd["q_nope"]), P(pfd["q_pe"]), P(pfd["kv_cache"]), P(pfd["pe_cache"]),
                                       P(pfd["cache_slot"]), P(pfd["end_pos"]), P(pfd["topk_idx"]), P(pfd["wkv_b"]),
                                       ctypes.c_float(pfd["scale"]), P(pf_out), R_pf, K_pf, S_pf, 1, P(pf_ws),
                                       pf_ws.numel(), None, None, sv)
 
-    t_prefill = time_kernel(k_prefill, 5)
+    t_prefill = time_graph(k_prefill, 5)
     del pfd, pf_out, pf_ws
 
-    # ---- end to end through the public API with host buffers
-    e2e = None
-    if rank == 0 or world > 1:
-        import sparse_latent_attention_absorb_b200 as api
-        # Per step one call of the C ABI's host-buffer entry point (through
-        # the Python binding): the step's queries, end positions and indices
-        # are uploaded from pinned host memory, the decode runs, the result is
-        # read back to pinned host memory, all on the call's stream.  Steps
-        # alternate between two streams, each with its own workspace, so the
-        # copies of one step overlap the kernels of the next.
-        names = ("q_nope", "q_pe", "end_pos", "topk_idx")
-        hins = [{k: s_["host"][k].contiguous().pin_memory() for k in names} for s_ in sets]
-        houts = [torch.empty((B, 128, 128), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-        hws = [torch.empty(api.host_workspace_size(B, K, S_max), dtype=torch.uint8, device=device) for _ in range(2)]
-        e2e_streams = [stream, torch.cuda.Stream(device=device)]
-        h2d = sum(hins[0][k].numel() * hins[0][k].element_size() for k in names)
-        d2h = houts[0].numel() * houts[0].element_size()
-
-        def e2e_step(i):
-            k, si = i % 2, i % NSETS
-            h = hins[si]
-            api.mla_sparse_decode_host(h["q_nope"], h["q_pe"], h["end_pos"], h["topk_idx"], sets[si]["kv_cache"],
-                                       sets[si]["pe_cache"], sets[si]["wkv_b"], sets[si]["scale"], houts[k], hws[k],
-                                       stream=e2e_streams[k])
-
-        for it in range(max(50, args.warmup)):  # host-side paths warm as well
-            e2e_step(it)
-        torch.cuda.synchronize()
-        barrier()
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        side_done = torch.cuda.Event()
-        f0.record(e2e_streams[0])
-        e2e_streams[1].wait_event(f0)
-        h0 = time.perf_counter()
-        for it in range(args.steps):
-            e2e_step(it)
-        host_ms = (time.perf_counter() - h0) * 1e3
-        side_done.record(e2e_streams[1])
-        e2e_streams[0].wait_event(side_done)
-        f1.record(e2e_streams[0])
-        torch.cuda.synchronize()
-        e_ms = f0.elapsed_time(f1)
-        print(f"e2e: {args.steps} steps, host enqueue {host_ms:.1f} ms, device {e_ms:.1f} ms", file=sys.stderr)
-        e_ms = max_over_ranks(e_ms, world, device)
-        e2e = {"value": whole_job_rate(B, world, args.steps, e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h,
-               "how": "per step one mla_sparse_decode_host call (pinned host inputs uploaded, decode, result read "
-                      "back on the call's stream); steps alternate between two streams"}
-
-    # ---- roofline of the dominant kernel and of the whole call
-    hbm, tf, tf_sus, kind = peaks()
-    sum_k = statistics.mean(s["sum_k"] for s in sets)
-    a_bytes = attend_bytes(B, K, sum_k)
-    achieved = a_bytes / (t_attend * 1e-3) / 1e9
-    traffic = ncu_traffic(args.workload)
-    call_bytes, call_flops = algorithmic(B, K, sum_k)
-    t_hbm = call_bytes / (hbm * 1e9)
-    t_tc = call_flops / (tf * 1e12)
-    roof_ms = max(t_hbm, t_tc) * 1e3
-
-    res = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "B": B, "heads": 128, "S_max": S_max, "K": K,
-                   "end_pos": list(w.end_pos), "index": w.index, "sum_k_mean": sum_k, "splits": n_split,
-                   "parallelism": f"replicas x{world} (batch rows)",
-                   "l2": f"{NSETS} rotating input sets (queries, indices, wkv_b copy each); per-step footprint "
-                         f"{call_bytes / 1e6:.0f} MB > 126 MB L2",
-                   "timing": "CUDA graphs of 4 consecutive steps (one per input set), CUDA events on the launching stream"},
-        "roofline": {"bound": "hbm", "kernel": "sparse_attend_kernel", "achieved": achieved, "peak": hbm,
-                     "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
-                     "peak_source": f"{kind} hbm_gbs", "alg_bytes_per_launch": a_bytes,
-                     "ms_per_launch": t_attend},
-        "call_roofline": {"alg_bytes": call_bytes, "alg_flops": call_flops, "t_hbm_ms": t_hbm * 1e3,
-                          "t_tensor_ms": t_tc * 1e3, "roofline_ms": roof_ms, "frac": roof_ms / ms_per_step,
-                          "bound": "hbm" if t_hbm >= t_tc else "tensor",
-                          "peaks": {"hbm_gbs": hbm, "bf16_tflops": tf, "source": kind}},
-        "kernels_ms": {"absorb": t_absorb, "sparse_attend": t_attend, "combine_value_up": t_combine},
+    extras = {
         "projection": {"what": "output projection delta = x . wo^T of the decode outputs, wo bf16 [7168, 16384]",
                        "ms_per_call": t_project, "launches_per_call": 1 if p_ws.numel() <= 256 else 2,
                        "roofline": {"bound": "hbm", "achieved": p_bytes / (t_project * 1e-3) / 1e9, "peak": hbm,
                                     "unit": "GB/s", "frac": p_bytes / (t_project * 1e-3) / 1e9 / hbm,
-                                    "alg_bytes_per_call": p_bytes, "peak_source": f"{kind} hbm_gbs"}},
+                                    "alg_bytes_per_call": p_bytes, "peak_source": "measured hbm_gbs"}},
         "prefill": {"what": "sparse prefill of one 4096-position sequence, top-2048, causal: one row per query "
                             "position (mla_sparse_prefill)", "ms_per_call": t_prefill,
                     "tokens_per_s": R_pf / (t_prefill * 1e-3), "selected_positions": pf_sel,
                     "gathered_GBps": pf_sel * 1152 / (t_prefill * 1e-3) / 1e9},
-        "gpu_launches": launches,
-        "e2e": e2e,
-        "clocks": clocks.summary(),
     }
-    for g in graphs:
-        del g
-    return res, base
+
+    # ---- end to end through the public API with host buffers
+    extras["e2e"] = e2e_measurement(args, dec, sets, w, device, stream, world)
+
+    # ---- every configuration of the pages, each with its own roofline
+    extras["per_config"] = per_config(lib, device, stream)
+    return extras
+
+
+def e2e_measurement(args, dec, sets, w, device, stream, world, n_streams=3):
+    """Per step one call of the C ABI's host-buffer entry point (through the
+    Python binding): the step's queries, end positions and indices are
+    uploaded from pinned host memory, the decode runs and the result is read
+    back to pinned host memory, all on the call's stream.  Steps rotate over
+    n_streams streams, each with its own workspace and output buffer, so the
+    uploads and read-backs of neighbouring steps overlap this step's kernels."""
+    import sparse_latent_attention_absorb_b200 as api
+    B, K, S_max = w.B, w.K, w.S_max
+    names = ("q_nope", "q_pe", "end_pos", "topk_idx")
+    hins = [{k: s_["host"][k].contiguous().pin_memory() for k in names} for s_ in sets]
+    houts = [torch.empty((B, 128, 128), dtype=torch.bfloat16).pin_memory() for _ in range(n_streams)]
+    hws = [torch.empty(api.host_workspace_size(B, K, S_max), dtype=torch.uint8, device=device)
+           for _ in range(n_streams)]
+    streams = [stream] + [torch.cuda.Stream(device=device) for _ in range(n_streams - 1)]
+    h2d = sum(hins[0][k].numel() * hins[0][k].element_size() for k in names)
+    d2h = houts[0].numel() * houts[0].element_size()
+
+    def step(i):
+        k, si = i % n_streams, i % len(sets)
+        h = hins[si]
+        api.mla_sparse_decode_host(h["q_nope"], h["q_pe"], h["end_pos"], h["topk_idx"], sets[si]["kv_cache"],
+                                   sets[si]["pe_cache"], sets[si]["wkv_b"], sets[si]["scale"], houts[k], hws[k],
+                                   stream=streams[k])
+
+    def window(n):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(streams[0])
+        for s_ in streams[1:]:
+            s_.wait_event(f0)
+        for it in range(n):
+            step(it)
+        for s_ in streams[1:]:
+            done = torch.cuda.Event()
+            done.record(s_)
+            streams[0].wait_event(done)
+        f1.record(streams[0])
+        torch.cuda.synchronize()
+        return f0.elapsed_time(f1)
+
+    for it in range(max(50, args.warmup)):  # host-side paths warm as well
+        step(it)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    probe = max_over_ranks(window(args.steps), world, device)
+    repeats = max(1, min(10000, math.ceil(500.0 / max(probe, 1e-3))))
+    wins = [max_over_ranks(window(args.steps), world, device) for _ in range(repeats)]
+    e_ms = statistics.median(wins)
+    return {"value": whole_job_rate(B, world, args.steps, e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "windows": repeats,
+            "how": f"per step one mla_sparse_decode_host call (pinned host inputs uploaded, decode, result read "
+                   f"back on the call's stream); steps rotate over {n_streams} streams; median of {repeats} "
+                   f"windows of {args.steps} steps"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -576,13 +732,16 @@ def reference_arm(args, rank, world, budget_s=90.0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    # ~0.15 s of timed steps by default: long enough for NVML to sample the
-    # clocks inside the region many times
-    ap.add_argument("--steps", type=int, default=2000)
+    # a window of 200 steps (~14 ms); windows repeat until they span 0.5 s
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.ALL_WORKLOADS))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="time the headline decode and its kernels only (no other configurations, projection, "
+                         "prefill, end-to-end or CPU baseline): a small footprint for profiler captures")
+    ap.add_argument("--sets", type=int, default=0, help="rotating input sets (default: enough to exceed 2x L2)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -604,7 +763,7 @@ def main():
     torch.cuda.set_device(device)
     res, base = gpu_arm(args, rank, world, device)
     if rank == 0:
-        if not args.no_cpu_baseline:
+        if not (args.no_cpu_baseline or args.no_extras):
             res["cpu_baseline"] = cpu_baseline(args, base["host"] if "host" in base else base)
         print(json.dumps(res), flush=True)
     if world > 1:

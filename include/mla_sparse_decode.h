@@ -32,12 +32,18 @@
  *     synchronisation happens.  An argument error is returned BEFORE anything
  *     is launched.  A launch error returns MLA_ERR_CUDA.  Faults during
  *     execution appear at the caller's next synchronisation; a device wait
- *     that exceeds its time limit writes MLA_ERR_DEVICE_TIMEOUT to *d_status
- *     (when d_status is not NULL) and the kernels return without hanging.
+ *     that exceeds its time limit (2 s; a healthy wait lasts microseconds)
+ *     writes MLA_ERR_DEVICE_TIMEOUT to *d_status (when d_status is not NULL)
+ *     and the kernels return without hanging, leaving the output incomplete.
+ *     With d_status NULL such a call cannot be told apart from a good one,
+ *     so production callers should pass a status word and check it.
  *   - Index semantics: topk_idx[b, k] selects cache position t of batch row b
  *     when 0 <= t < min(end_pos[b], S_max); any other value (canonically -1)
  *     is padding and is skipped.  Valid indices of one row must be distinct
- *     (the indexer's top-k output is); a repeated index would be counted twice.
+ *     (the indexer's top-k output is): the pages' mask scatters 0 into a -inf
+ *     row, so a repeat selects a position once, but the kernels gather every
+ *     listed entry and would count a repeat twice.  mla_check_topk_indices
+ *     (or mla_set_index_checks) reports rows that break this.
  *     Index order is irrelevant.  A row with no valid index yields out = 0 and
  *     lse = -inf.
  *   - Batch row b reads cache slot b (the excerpt slices kv_cache[:bsz]);
@@ -66,7 +72,7 @@ typedef enum {
   MLA_ERR_WORKSPACE = 2,      /* workspace missing, misaligned or too small */
   MLA_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed       */
   MLA_ERR_DEVICE_TIMEOUT = 4, /* written to *d_status by a timed-out wait   */
-  MLA_ERR_BAD_INDEX = 5,      /* reserved for index validation reports      */
+  MLA_ERR_BAD_INDEX = 5,      /* written to *d_status: a repeated index     */
   MLA_ERR_UNSUPPORTED = 6     /* device is not sm_100                       */
 } mla_status;
 
@@ -151,6 +157,34 @@ int mla_sparse_attend(const void* q_lat, const void* q_pe, const void* kv_cache,
  */
 int mla_combine_value_up(const void* o_part, const float* lse_part, const void* wkv_b, void* out,
                          float* lse_out, int B, int n_split, cudaStream_t stream);
+
+/*
+ * Index validation (the index mask of model.py 601-602 on the page "Query-key
+ * similarity": a -inf row with 0 scattered at the selected positions, so each
+ * position is selected at most once).  One CTA per row marks the row's valid
+ * entries (0 <= t < min(end_pos[b], S_max); the rest is padding) in a bitmap
+ * and finds any entry listed twice.
+ *   end_pos, topk_idx  as in mla_sparse_decode (device, 16-byte aligned)
+ *   d_status     optional device int: receives MLA_ERR_BAD_INDEX (if it still
+ *                holds 0) when some row has a repeated valid entry
+ *   d_row_flags  optional device int [B]: 1 for a row with a repeat, else 0
+ * At least one of d_status, d_row_flags must be given.  Enqueued on `stream`;
+ * reads B*K indices once per 1,048,576 positions of end_pos.  The decode
+ * itself does not depend on the result.  Returns an mla_status.
+ */
+int mla_check_topk_indices(const int32_t* end_pos, const int32_t* topk_idx, int B, int K, int S_max,
+                           int* d_status, int* d_row_flags, cudaStream_t stream);
+
+/*
+ * Opt-in debug mode for the whole process: with enable != 0, every call of
+ * mla_sparse_decode, mla_sparse_prefill and the entry points built on them
+ * (noalloc, host-buffer, decode + projection) that is given a d_status
+ * first enqueues mla_check_topk_indices on its index rows, so a repeated
+ * index ends up as MLA_ERR_BAD_INDEX in *d_status (the decode still runs).
+ * Off by default; costs one extra kernel per call.  Returns the previous
+ * setting.
+ */
+int mla_set_index_checks(int enable);
 
 /*
  * Size of the library's fixed device scratch used by

@@ -27,7 +27,7 @@ EXPORTS = ("mla_status_string", "mla_num_splits", "mla_sparse_decode_workspace_s
            "mla_sparse_decode_host_workspace_size", "mla_sparse_decode_host",
            "mla_output_projection_workspace_size", "mla_output_projection",
            "mla_sparse_decode_project_workspace_size", "mla_sparse_decode_project", "mla_sparse_prefill",
-           "mla_selftest_wait_timeout")
+           "mla_selftest_wait_timeout", "mla_check_topk_indices", "mla_set_index_checks")
 STATIC_SCRATCH_BYTES = 32 << 20  # MLA_STATIC_SCRATCH_BYTES
 
 _lib = None
@@ -78,6 +78,10 @@ def load_library():
     lib.mla_sparse_decode_project.argtypes = [p, p, p, p, p, p, p, f, p, p, i, i, i, i, p, sz, p, p, p]
     lib.mla_sparse_prefill.restype = i
     lib.mla_sparse_prefill.argtypes = [p, p, p, p, p, p, p, p, f, p, i, i, i, i, p, sz, p, p, p]
+    lib.mla_check_topk_indices.restype = i
+    lib.mla_check_topk_indices.argtypes = [p, p, i, i, i, p, p, p]
+    lib.mla_set_index_checks.restype = i
+    lib.mla_set_index_checks.argtypes = [i]
     lib.mla_selftest_wait_timeout.restype = i
     lib.mla_selftest_wait_timeout.argtypes = [p, p, p]
     _lib = lib
@@ -413,3 +417,30 @@ def selftest_wait_timeout(stream=None):
     _raise(lib.mla_selftest_wait_timeout(_ptr(status), _ptr(result), _stream(stream)), "mla_selftest_wait_timeout")
     torch.cuda.synchronize()
     return int(status.item()), int(result.item())
+
+
+def mla_check_topk_indices(end_pos, topk_idx, S_max: int, d_status=None, row_flags=None, stream=None):
+    """Repeated valid entries of the index rows (mla_check_topk_indices).
+    Writes MLA_ERR_BAD_INDEX into d_status (int32 [1], if it holds 0) and 1/0
+    per row into row_flags (int32 [B]); allocates row_flags when both are
+    None.  Returns row_flags (or None)."""
+    lib = load_library()
+    B, K = topk_idx.shape
+    _check(end_pos, "end_pos", torch.int32, (B,))
+    _check(topk_idx, "topk_idx", torch.int32)
+    if d_status is None and row_flags is None:
+        row_flags = torch.empty(B, dtype=torch.int32, device=topk_idx.device)
+    if row_flags is not None:
+        _check(row_flags, "row_flags", torch.int32, (B,))
+    if d_status is not None:
+        _check(d_status, "d_status", torch.int32)
+    rc = lib.mla_check_topk_indices(_ptr(end_pos), _ptr(topk_idx), B, K, S_max, _ptr(d_status), _ptr(row_flags),
+                                    _stream(stream))
+    _raise(rc, "mla_check_topk_indices")
+    return row_flags
+
+
+def set_index_checks(enable: bool) -> bool:
+    """Turns the process-wide opt-in index validation on or off
+    (mla_set_index_checks); returns the previous setting."""
+    return bool(load_library().mla_set_index_checks(1 if enable else 0))

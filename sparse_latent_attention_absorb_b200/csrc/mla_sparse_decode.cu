@@ -11,6 +11,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "index_check.cuh"
 #include "kernels.cuh"
 #include "mla_sparse_decode.h"
 #include "projection.cuh"
@@ -55,7 +56,9 @@ int current_device(DeviceInfo** info) {
       if (cudaFuncSetAttribute(absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAbsorbSmemBytes) != cudaSuccess ||
           cudaFuncSetAttribute(sparse_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttendSmemBytes) != cudaSuccess ||
           cudaFuncSetAttribute(combine_value_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCombineSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(projection_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, proj_smem_max()) != cudaSuccess)
+          cudaFuncSetAttribute(projection_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, proj_smem_max()) != cudaSuccess ||
+          cudaFuncSetAttribute(check_indices_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kCheckMaxWords * 4) != cudaSuccess)
         return MLA_ERR_CUDA;
     }
     d.configured = true;
@@ -436,6 +439,19 @@ extern "C" int mla_combine_value_up(const void* o_part, const float* lse_part, c
 }
 
 namespace {
+// Opt-in index validation before every decode / prefill call (see
+// mla_set_index_checks); off by default.
+std::atomic<int> g_index_checks{0};
+
+int launch_check_indices(const int32_t* end_pos, const int32_t* topk_idx, int B, int K, int S_max, int* d_status,
+                         int* d_dup, cudaStream_t stream) {
+  const size_t smem = (size_t)check_bitmap_words(S_max) * 4;
+  return launch_ex(check_indices_kernel, dim3((unsigned)B), dim3(kCheckThreads), smem, stream, false, end_pos,
+                   topk_idx, K, S_max, d_status, d_dup);
+}
+}  // namespace
+
+namespace {
 // The three kernels over B rows: row b is one query (its q_nope, q_pe, index
 // row and end position) and reads cache slot cache_slot[b], or b when
 // cache_slot is null.  Shared by the decode step (a row per batch row) and
@@ -463,6 +479,9 @@ int run_rows(const void* q_nope, const void* q_pe, const void* kv_cache, const v
   void* o_part = ws + wl.o_part;
   float* lse_part = reinterpret_cast<float*>(ws + wl.lse_part);
 
+  if (d_status && g_index_checks.load(std::memory_order_relaxed) &&
+      (rc = launch_check_indices(end_pos, topk_idx, B, K, S_max, d_status, nullptr, stream)) != MLA_OK)
+    return rc;
   // The attention and combine kernels depend programmatically on the kernel
   // before them: each starts while its predecessor drains and waits for it
   // only where it reads that kernel's output.  The absorption kernel is an
@@ -496,6 +515,24 @@ extern "C" int mla_sparse_prefill(const void* q_nope, const void* q_pe, const vo
   if (!cache_slot || !aligned16(cache_slot) || n_slots < 1) return MLA_ERR_INVALID_ARG;
   return run_rows(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, scale, out, R, K, S_max, cache_slot,
                   n_slots, workspace, workspace_bytes, lse_out, d_status, stream);
+}
+
+// Index validation (see the header): repeated valid entries of a row.
+extern "C" int mla_check_topk_indices(const int32_t* end_pos, const int32_t* topk_idx, int B, int K, int S_max,
+                                      int* d_status, int* d_row_flags, cudaStream_t stream) {
+  if (!end_pos || !topk_idx || !aligned16(end_pos) || !aligned16(topk_idx)) return MLA_ERR_INVALID_ARG;
+  if (!d_status && !d_row_flags) return MLA_ERR_INVALID_ARG;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (d_row_flags && (reinterpret_cast<uintptr_t>(d_row_flags) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (!sizes_ok(B, K, S_max)) return MLA_ERR_INVALID_ARG;
+  DeviceInfo* info = nullptr;
+  int rc = prepare(&info);
+  if (rc != MLA_OK) return rc;
+  return launch_check_indices(end_pos, topk_idx, B, K, S_max, d_status, d_row_flags, stream);
+}
+
+extern "C" int mla_set_index_checks(int enable) {
+  return g_index_checks.exchange(enable ? 1 : 0);
 }
 
 #ifdef MLA_TRACE

@@ -104,7 +104,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 // kWaitLimitNs sets the CTA's abort flag, records MLA_ERR_DEVICE_TIMEOUT in the
 // caller's status word (if any) and returns false; once a CTA is aborting all
 // further waits return at once, so every thread reaches the kernel's exit path
-// (TMEM release, cluster barrier) instead of hanging.
+// (TMEM release, cluster barrier) instead of hanging.  The out-of-line helpers
+// are static: each translation unit that includes this header has its own.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s; a healthy wait is < 1 ms
 
 struct AbortState {
@@ -112,7 +113,7 @@ struct AbortState {
   int* status;         // caller's device status word, may be null
 };
 
-__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, AbortState ab, bool cluster_scope) {
+static __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, AbortState ab, bool cluster_scope) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 0;; ++it) {
     bool ok = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
@@ -142,7 +143,7 @@ __device__ __forceinline__ bool wait_cluster(uint32_t bar, uint32_t parity, Abor
 
 // Bounded wait until a shared-memory counter written by another thread of
 // this CTA reaches `target` (a scheduling condition: no data is handed over).
-__device__ __noinline__ bool wait_counter_slow(const volatile int* counter, int target, AbortState ab) {
+static __device__ __noinline__ bool wait_counter_slow(const volatile int* counter, int target, AbortState ab) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 0;; ++it) {
     if (*counter >= target) return true;

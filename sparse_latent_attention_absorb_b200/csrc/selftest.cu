@@ -8,14 +8,9 @@
 #include <cstdint>
 
 #include "mla_sparse_decode.h"
-
-// The inline-PTX layer, with internal linkage in this translation unit: its
-// out-of-line helpers (wait_slow and friends) are also compiled into the
-// decode's translation unit, and the two copies must not collide at link
-// time.  Same source, same wait().
-namespace {
+// The inline-PTX layer (its out-of-line helpers are static: this translation
+// unit and the decode's each hold their own copy of the same wait()).
 #include "ptx.cuh"
-}
 
 namespace {
 

@@ -197,3 +197,33 @@ def test_prefill_rejects_bad_arguments_without_a_launch(lib):
     assert call(R=0) == INVALID_ARG
     assert call(K=0) == INVALID_ARG
     assert call(scale=float("inf")) == INVALID_ARG
+
+
+def test_index_check_rejects_bad_arguments_without_a_launch(lib):
+    A = 0x10000
+    st = _fake(A)
+
+    def call(ep=_fake(A), idx=_fake(A), B=2, K=16, S=32, status=st, flags=None):
+        return lib.mla_check_topk_indices(ep, idx, B, K, S, status, flags, None)
+
+    assert call(ep=None) == INVALID_ARG
+    assert call(idx=None) == INVALID_ARG
+    assert call(ep=_fake(A + 4)) == INVALID_ARG
+    assert call(idx=_fake(A + 8)) == INVALID_ARG
+    assert call(status=None, flags=None) == INVALID_ARG  # nothing to report into
+    assert call(status=_fake(A + 2)) == INVALID_ARG
+    assert call(status=None, flags=_fake(A + 1)) == INVALID_ARG
+    assert call(B=0) == INVALID_ARG
+    assert call(K=0) == INVALID_ARG
+    assert call(S=0) == INVALID_ARG
+
+
+def test_index_check_flag_is_a_process_wide_switch(lib):
+    # a host-side flag only: nothing is launched
+    prev = lib.mla_set_index_checks(1)
+    try:
+        assert lib.mla_set_index_checks(1) == 1
+        assert lib.mla_set_index_checks(0) == 1
+        assert lib.mla_set_index_checks(0) == 0
+    finally:
+        lib.mla_set_index_checks(prev)

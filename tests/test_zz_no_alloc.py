@@ -26,7 +26,10 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-@pytest.mark.parametrize("name", ["small_b4_ctx600-2k_recent128_top400", "b8_ctx4096_top2048"])
+# the last case is the largest configuration the fixed scratch is sized for
+# (B = 64 rows, K = 2048)
+@pytest.mark.parametrize("name", ["small_b4_ctx600-2k_recent128_top400", "b8_ctx4096_top2048",
+                                  "b64_ctx1k-32k_top2048"])
 def test_noalloc_matches_allocating_entry_point_twice(name):
     lib = pkg.load_library()
     d = wl.generate(name)
