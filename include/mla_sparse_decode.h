@@ -2,9 +2,12 @@
  * mla_sparse_decode.h -- C ABI of the B200 (sm_100a) sparse MLA decode library.
  *
  * Also declared here, after the decode step: the sparse prefill over the same
- * kernels (mla_sparse_prefill, page "Queries") and the attention output
+ * kernels (mla_sparse_prefill, page "Queries"), the attention output
  * projection (mla_output_projection, mla_sparse_decode_project, page
- * "Attention update").
+ * "Attention update"), a tensor-parallel shard of both
+ * (mla_sparse_decode_heads, mla_output_projection_shard), the fp8 weight
+ * dequantisation (mla_dequant_fp8_blocks) and index validation
+ * (mla_check_topk_indices).
  *
  * One decode step of DeepSeek-V3.2-Exp's absorbed multi-head latent attention
  * with the indexer's top-k mask, as the atlas pages of
@@ -320,6 +323,74 @@ int mla_sparse_decode_project(const void* q_nope, const void* q_pe, const void* 
                               const int32_t* end_pos, const int32_t* topk_idx, const void* wkv_b, float scale,
                               const void* wo, void* delta, int B, int K, int S_max, int dim, void* workspace,
                               size_t workspace_bytes, float* lse_out, int* d_status, cudaStream_t stream);
+
+/*
+ * fp8 weights (the decode excerpt on the page "Query-key similarity",
+ * model.py 591-592: when wkv_b is stored in fp8 with a scale, the decode
+ * first builds self.dequant_wkv_b = weight_dequant(wkv_b.weight, wkv_b.scale)
+ * once and uses it in place of wkv_b from then on).  The pages do not print
+ * the format; this entry point reads it as DeepSeek-V3's block format:
+ *   w_fp8   OCP FP8 E4M3 codes [rows, cols] (1 byte each)
+ *   scale   f32 [ceil(rows/128), ceil(cols/128)]: one scale per 128 x 128 block
+ *   w_bf16  bf16 [rows, cols]:
+ *           w_bf16[r,c] = bf16( e4m3(w_fp8[r,c]) * scale[r/128, c/128] ),
+ *           the product exact and rounded once to nearest (ties to even)
+ * For wkv_b: rows = 128*256 (n_heads*256 for a shard), cols = 512, scale
+ * [256, 4].  The result is the bf16 wkv_b every decode entry point takes, so
+ * a caller holding fp8 weights dequantises once, as the pages do, and keeps
+ * the result.  cols must be a multiple of 16; w_fp8 and w_bf16 16-byte
+ * aligned, scale 4-byte aligned.  Enqueued on `stream`.  Returns an
+ * mla_status.
+ */
+int mla_dequant_fp8_blocks(const void* w_fp8, const float* scale, void* w_bf16, int rows, int cols,
+                           cudaStream_t stream);
+
+/*
+ * Tensor parallelism, one shard (the MLA constructor excerpt on the page
+ * "Queries", model.py 523-539: wkv_b is a ColumnParallelLinear, so a rank
+ * holds n_local_heads = 128 / world_size heads and views its wkv_b rows as
+ * [n_local_heads, 256, 512]; wo is a RowParallelLinear whose partial outputs
+ * the ranks sum).  The decode step for n_heads consecutive heads:
+ *   q_nope bf16 [B,n_heads,128], q_pe bf16 [B,n_heads,64]  the shard's heads
+ *   wkv_b  bf16 [n_heads*256,512]  the shard's rows of wkv_b
+ *   out    bf16 [B,n_heads,128],  lse_out f32 [B,n_heads] (optional)
+ *   kv_cache, pe_cache, end_pos, topk_idx, scale: as in mla_sparse_decode
+ *            (the latent cache and the index rows are shared by all heads,
+ *            so every shard holds them whole)
+ *   workspace: mla_sparse_decode_heads_workspace_size(B, K, S_max, n_heads)
+ * 1 <= n_heads <= 128; with n_heads = 128 this is mla_sparse_decode.  The
+ * attention kernel keeps the heads on the 128 lanes of its MMA tile: lanes
+ * past n_heads carry a zero query and store nothing, so a shard's attention
+ * costs as much as all 128 heads' (the weight-bound steps scale with
+ * n_heads).  Returns an mla_status; the size function returns 0 for invalid
+ * sizes.
+ */
+size_t mla_sparse_decode_heads_workspace_size(int B, int K, int S_max, int n_heads);
+int mla_sparse_decode_heads(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                            const int32_t* end_pos, const int32_t* topk_idx, const void* wkv_b, float scale,
+                            void* out, int B, int K, int S_max, int n_heads, void* workspace,
+                            size_t workspace_bytes, float* lse_out, int* d_status, cudaStream_t stream);
+
+/*
+ * The row-parallel partial of the output projection (wo = RowParallelLinear
+ * on the page "Queries"; the projection of the page "Attention update"):
+ *   delta_r[b, n] = bf16( sum_{k < k_in} x[b, k] * wo[n, k] )   (fp32 accumulate)
+ *   x      bf16 [B, k_in]    the shard's decode output [B,n_heads,128] flattened
+ *   wo     bf16 rows of ld_wo elements (16-byte aligned, ld_wo a multiple of
+ *          8 and >= k_in); columns [0, k_in) of each of the dim rows are used
+ *   delta  bf16 [B, dim]
+ *   k_in   a multiple of 64, 64 <= k_in <= 16384
+ *   workspace: mla_output_projection_shard_workspace_size(B, dim, k_in)
+ * For rank r of T ranks holding n_heads = 128 / T heads: x = its out,
+ * wo = the full wo + r*n_heads*128 (ld_wo = 16384) or its own column slice
+ * (ld_wo = k_in), k_in = n_heads*128.  Summing delta_r over the ranks (the
+ * all-reduce after the RowParallelLinear) gives the projection of all heads;
+ * with k_in = 16384 and ld_wo = 16384 this is mla_output_projection.
+ * Returns an mla_status; the size function returns 0 for invalid sizes.
+ */
+size_t mla_output_projection_shard_workspace_size(int B, int dim, int k_in);
+int mla_output_projection_shard(const void* x, const void* wo, long long ld_wo, void* delta, int B, int dim, int k_in,
+                                void* workspace, size_t workspace_bytes, int* d_status, cudaStream_t stream);
 
 /*
  * Self-test of the bounded waits every kernel relies on (no counterpart on the

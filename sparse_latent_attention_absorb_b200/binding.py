@@ -27,7 +27,9 @@ EXPORTS = ("mla_status_string", "mla_num_splits", "mla_sparse_decode_workspace_s
            "mla_sparse_decode_host_workspace_size", "mla_sparse_decode_host",
            "mla_output_projection_workspace_size", "mla_output_projection",
            "mla_sparse_decode_project_workspace_size", "mla_sparse_decode_project", "mla_sparse_prefill",
-           "mla_selftest_wait_timeout", "mla_check_topk_indices", "mla_set_index_checks")
+           "mla_selftest_wait_timeout", "mla_check_topk_indices", "mla_set_index_checks",
+           "mla_sparse_decode_heads_workspace_size", "mla_sparse_decode_heads",
+           "mla_output_projection_shard_workspace_size", "mla_output_projection_shard", "mla_dequant_fp8_blocks")
 STATIC_SCRATCH_BYTES = 32 << 20  # MLA_STATIC_SCRATCH_BYTES
 
 _lib = None
@@ -82,6 +84,16 @@ def load_library():
     lib.mla_check_topk_indices.argtypes = [p, p, i, i, i, p, p, p]
     lib.mla_set_index_checks.restype = i
     lib.mla_set_index_checks.argtypes = [i]
+    lib.mla_sparse_decode_heads_workspace_size.restype = sz
+    lib.mla_sparse_decode_heads_workspace_size.argtypes = [i, i, i, i]
+    lib.mla_sparse_decode_heads.restype = i
+    lib.mla_sparse_decode_heads.argtypes = [p, p, p, p, p, p, p, f, p, i, i, i, i, p, sz, p, p, p]
+    lib.mla_output_projection_shard_workspace_size.restype = sz
+    lib.mla_output_projection_shard_workspace_size.argtypes = [i, i, i]
+    lib.mla_dequant_fp8_blocks.restype = i
+    lib.mla_dequant_fp8_blocks.argtypes = [p, p, p, i, i, p]
+    lib.mla_output_projection_shard.restype = i
+    lib.mla_output_projection_shard.argtypes = [p, p, ctypes.c_longlong, p, i, i, i, p, sz, p, p]
     lib.mla_selftest_wait_timeout.restype = i
     lib.mla_selftest_wait_timeout.argtypes = [p, p, p]
     _lib = lib
@@ -444,3 +456,97 @@ def set_index_checks(enable: bool) -> bool:
     """Turns the process-wide opt-in index validation on or off
     (mla_set_index_checks); returns the previous setting."""
     return bool(load_library().mla_set_index_checks(1 if enable else 0))
+
+
+def mla_sparse_decode_heads(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, scale, out=None,
+                            workspace=None, lse_out=None, d_status=None, stream=None):
+    """One tensor-parallel shard of the decode step: the heads of q_nope
+    (bf16 [B, n_heads, 128]) with wkv_b holding their rows (bf16
+    [n_heads*256, 512]); returns ``out`` (bf16 [B, n_heads, 128])."""
+    lib = load_library()
+    B, n_heads = q_nope.shape[0], q_nope.shape[1]
+    S_max = kv_cache.shape[1]
+    K = topk_idx.shape[1]
+    bf = torch.bfloat16
+    _check(q_nope, "q_nope", bf, (B, n_heads, D_NOPE))
+    _check(q_pe, "q_pe", bf, (B, n_heads, D_ROPE))
+    _check(kv_cache, "kv_cache", bf, (B, S_max, D_LAT))
+    _check(pe_cache, "pe_cache", bf, (B, S_max, D_ROPE))
+    _check(end_pos, "end_pos", torch.int32, (B,))
+    _check(topk_idx, "topk_idx", torch.int32, (B, K))
+    _check(wkv_b, "wkv_b", bf, (n_heads * (D_NOPE + D_V), D_LAT))
+    if out is None:
+        out = torch.empty((B, n_heads, D_V), dtype=bf, device=q_nope.device)
+    _check(out, "out", bf, (B, n_heads, D_V))
+    if lse_out is not None:
+        _check(lse_out, "lse_out", torch.float32, (B, n_heads))
+    if workspace is None:
+        n = lib.mla_sparse_decode_heads_workspace_size(B, K, S_max, n_heads)
+        if n == 0:
+            raise MLAError(1, "mla_sparse_decode_heads_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q_nope.device)
+    _check(workspace, "workspace", torch.uint8)
+    rc = lib.mla_sparse_decode_heads(_ptr(q_nope), _ptr(q_pe), _ptr(kv_cache), _ptr(pe_cache), _ptr(end_pos),
+                                     _ptr(topk_idx), _ptr(wkv_b), float(scale), _ptr(out), B, K, S_max, n_heads,
+                                     _ptr(workspace), workspace.numel(), _ptr(lse_out), _ptr(d_status),
+                                     _stream(stream))
+    _raise(rc, "mla_sparse_decode_heads")
+    return out
+
+
+def mla_output_projection_shard(x, wo, delta=None, workspace=None, d_status=None, stream=None):
+    """Row-parallel partial of the output projection: x bf16 [B, k_in] (a
+    shard's flattened decode output), wo a bf16 [dim, k_in] view whose rows
+    may be strided (a column slice of the full wo); returns delta bf16
+    [B, dim] = x . wo^T."""
+    lib = load_library()
+    B, k_in = x.shape
+    dim = wo.shape[0]
+    _check(x, "x", torch.bfloat16, (B, k_in))
+    if not (wo.is_cuda and wo.dtype == torch.bfloat16 and wo.dim() == 2 and wo.shape[1] == k_in and wo.stride(1) == 1):
+        raise ValueError("wo: expected a CUDA bf16 [dim, k_in] view with unit column stride")
+    if delta is None:
+        delta = torch.empty((B, dim), dtype=torch.bfloat16, device=x.device)
+    _check(delta, "delta", torch.bfloat16, (B, dim))
+    if workspace is None:
+        n = lib.mla_output_projection_shard_workspace_size(B, dim, k_in)
+        if n == 0:
+            raise MLAError(1, "mla_output_projection_shard_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=x.device)
+    _check(workspace, "workspace", torch.uint8)
+    rc = lib.mla_output_projection_shard(_ptr(x), _ptr(wo), wo.stride(0), _ptr(delta), B, dim, k_in, _ptr(workspace),
+                                         workspace.numel(), _ptr(d_status), _stream(stream))
+    _raise(rc, "mla_output_projection_shard")
+    return delta
+
+
+def mla_dequant_fp8_blocks(w_fp8, scale, out=None, stream=None):
+    """bf16 weight from E4M3 codes (uint8 [rows, cols], or a float8_e4m3fn
+    tensor) and one f32 scale per 128 x 128 block; returns out (bf16
+    [rows, cols])."""
+    lib = load_library()
+    if w_fp8.dtype != torch.uint8:
+        w_fp8 = w_fp8.view(torch.uint8)
+    rows, cols = w_fp8.shape
+    _check(w_fp8, "w_fp8", torch.uint8, (rows, cols))
+    _check(scale, "scale", torch.float32, ((rows + 127) // 128, (cols + 127) // 128))
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.bfloat16, device=w_fp8.device)
+    _check(out, "out", torch.bfloat16, (rows, cols))
+    _raise(lib.mla_dequant_fp8_blocks(_ptr(w_fp8), _ptr(scale), _ptr(out), rows, cols, _stream(stream)),
+           "mla_dequant_fp8_blocks")
+    return out
+
+
+class Fp8Wkvb:
+    """wkv_b held in fp8 with block scales, dequantised to bf16 on first use
+    and kept (the decode excerpt's ``self.dequant_wkv_b``): ``weight()``
+    returns the bf16 wkv_b that every decode entry point takes."""
+
+    def __init__(self, w_fp8, scale):
+        self.w_fp8, self.scale, self._bf16 = w_fp8, scale, None
+
+    def weight(self, stream=None):
+        if self._bf16 is None:
+            self._bf16 = mla_dequant_fp8_blocks(self.w_fp8, self.scale, stream=stream)
+        return self._bf16

@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libmla_sparse_decode.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 SOURCES = [os.path.join(CSRC, "mla_sparse_decode.cu"), os.path.join(CSRC, "selftest.cu")]
-DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("kernels.cuh", "ptx.cuh", "projection.cuh", "projection_plan.h", "index_check.cuh")] + [
+DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("kernels.cuh", "ptx.cuh", "projection.cuh", "projection_plan.h", "index_check.cuh", "dequant.cuh")] + [
     os.path.join(INCLUDE, "mla_sparse_decode.h")]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]

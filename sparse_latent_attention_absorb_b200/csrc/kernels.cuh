@@ -38,7 +38,8 @@ __device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* p) {
 // =============================================================================
 // absorb_kernel: q_lat[b,h,c] = sum_d q_nope[b,h,d] * W_UK[h,d,c]
 //
-// Swap-AB GEMM per (head h, 128-column chunk of c, tile of up to 128 rows b):
+// Swap-AB GEMM per (head h, 128-column chunk of c, tile of up to 128 rows b),
+// over the n_heads heads of the call (128, or a tensor-parallel shard's):
 //   D[c, b] = sum_d W_UK[h, d, c] * q_nope[b, h, d]
 // M = 128 (c), N = batch tile (multiple of 16), K = 128 (d).
 // A = W_UK[h][:, chunk] is M-major in memory (c contiguous): two TMA boxes of
@@ -54,7 +55,7 @@ constexpr int kAbsorbSmemBytes = absorb_smem_bytes(kAbsorbNMax);
 
 __global__ void __launch_bounds__(128, 1)
 absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
-              __nv_bfloat16* __restrict__ q_lat, int B, int n_tile, int* d_status) {
+              __nv_bfloat16* __restrict__ q_lat, int B, int n_tile, int n_heads, int* d_status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -124,7 +125,7 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const int b = b0 + n0 + j;
-      if (b < B) q_lat[((size_t)b * kH + h) * kDl + c] = __float2bfloat16_rn(__uint_as_float(v[j]));
+      if (b < B) q_lat[((size_t)b * n_heads + h) * kDl + c] = __float2bfloat16_rn(__uint_as_float(v[j]));
     }
   }
   tc_fence_before();
@@ -314,7 +315,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
                      const int32_t* __restrict__ end_pos, const int32_t* __restrict__ topk_idx, float scale,
                      void* __restrict__ o_part, float* __restrict__ lse_part, int K, int S_max, int n_split,
                      int span, const __nv_bfloat16* __restrict__ w_next, const int32_t* __restrict__ cache_slot,
-                     int n_slots, int* d_status) {
+                     int n_slots, int n_heads, int* d_status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -470,7 +471,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     // warp 0 pulls W_UV of head blockIdx.x (+ gridDim.x ...) into L2 for the
     // value-up kernel that follows (w_next = wkv_b, or null to skip).
     if (g == 0 && lane == 0 && w_next != nullptr) {
-      for (int hh = blockIdx.x; hh < kH; hh += gridDim.x) {
+      for (int hh = blockIdx.x; hh < n_heads; hh += gridDim.x) {
         const __nv_bfloat16* w = w_next + (size_t)(hh * kHeadRows + kDn) * kDl;  // 128 rows x 512: 128 KB
 #pragma unroll
         for (int part = 0; part < 4; ++part) prefetch_l2(w + part * 32 * kDl, 32 * kDl * 2);
@@ -542,7 +543,8 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     // ------------------------------------------------------------ softmax
     const int grp = warp >> 2;      // tiles grp, grp+2, ...
     const int qd = warp & 3;        // TMEM lane quarter
-    const int i = qd * 32 + lane;   // head
+    const int i = qd * 32 + lane;   // head (TMEM lane)
+    const bool live = i < n_heads;  // lanes past the call's heads hold a zero query and write nothing
     const bool leader = (qd == 0 && lane == 0);
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
 
@@ -551,13 +553,13 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     // memory as a 64B-swizzled K-major row.
     {
       grid_dep_wait();  // q_lat comes from the absorption kernel
-      const uint4* ql = reinterpret_cast<const uint4*>(q_lat + ((size_t)b * kH + i) * kDl + rank * 256);
+      const uint4* ql = reinterpret_cast<const uint4*>(q_lat + ((size_t)b * n_heads + (live ? i : 0)) * kDl + rank * 256);
 #pragma unroll
       for (int part = 0; part < 2; ++part) {  // 64 latent values = 32 columns each
         uint32_t r[32];
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
-          const uint4 x = __ldg(ql + (2 * grp + part) * 8 + v);
+          const uint4 x = live ? __ldg(ql + (2 * grp + part) * 8 + v) : make_uint4(0u, 0u, 0u, 0u);
           r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
         }
         tmem_st32(tmem + lane_base + kColQ + (2 * grp + part) * 32, r);
@@ -565,10 +567,10 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       tmem_wait_st();
       tc_fence_before();
       if (grp == 1) {
-        const uint4* qp = reinterpret_cast<const uint4*>(q_pe + ((size_t)b * kH + i) * kDr + rank * 32);
+        const uint4* qp = reinterpret_cast<const uint4*>(q_pe + ((size_t)b * n_heads + (live ? i : 0)) * kDr + rank * 32);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          const uint4 x = __ldg(qp + v);
+          const uint4 x = live ? __ldg(qp + v) : make_uint4(0u, 0u, 0u, 0u);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sQpe + sw64_offset(i, v)), "r"(x.x),
                        "r"(x.y), "r"(x.z), "r"(x.w)
                        : "memory");
@@ -790,7 +792,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
     // A row of one split is final here: its mixed latent O~ goes out in bf16
     // (the value-up operand); several splits keep f32 partials for the merge.
-    const size_t orow = (((size_t)b * n_split + split) * kH + i) * kDl + rank * 256 + 128 * grp;
+    const size_t orow = (((size_t)b * n_split + split) * n_heads + (live ? i : 0)) * kDl + rank * 256 + 128 * grp;
 #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {
       uint32_t ov[32];
@@ -801,7 +803,9 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
 #pragma unroll
         for (int t = 0; t < 32; ++t) ov[t] = 0u;
       }
-      if (n_split == 1) {
+      if (!live) {
+        // nothing to store for a lane past the call's heads
+      } else if (n_split == 1) {
         __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(o_part) + orow + cc * 32;
 #pragma unroll
         for (int t = 0; t < 32; t += 8) {
@@ -821,8 +825,8 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
         }
       }
     }
-    if (rank == 0 && grp == 0) {
-      lse_part[((size_t)b * n_split + split) * kH + i] =
+    if (rank == 0 && grp == 0 && live) {
+      lse_part[((size_t)b * n_split + split) * n_heads + i] =
           l_sum > 0.f ? (m_fin + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
     }
   }
@@ -864,7 +868,7 @@ __global__ void __launch_bounds__(kCombineThreads, 1)
 combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_o,
                         const void* __restrict__ o_part, const float* __restrict__ lse_part,
                         __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out, int B, int n_split, int n_tile,
-                        int* d_status) {
+                        int n_heads, int* d_status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -917,24 +921,25 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
       tma_prefetch_desc(&tm_o);
       for (int kb = 0; kb < 8; ++kb) tma_load_3d(sB + kb * n_tile * 128, &tm_o, bar_k(kb), kb * 64, h, b0);
     }
-    if (tid < rows && lse_out) lse_out[(size_t)(b0 + tid) * kH + h] = lse_part[(size_t)(b0 + tid) * kH + h];
+    if (tid < rows && lse_out)
+      lse_out[(size_t)(b0 + tid) * n_heads + h] = lse_part[(size_t)(b0 + tid) * n_heads + h];
   } else {
     const float* o_f32 = static_cast<const float*>(o_part);
     // split weights, one row per thread
     if (tid < rows) {
       const int b = b0 + tid;
       float mx = -INFINITY;
-      for (int s = 0; s < n_split; ++s) mx = fmaxf(mx, lse_part[((size_t)b * n_split + s) * kH + h]);
+      for (int s = 0; s < n_split; ++s) mx = fmaxf(mx, lse_part[((size_t)b * n_split + s) * n_heads + h]);
       float total = 0.f;
       for (int s = 0; s < n_split; ++s) {
-        const float l = lse_part[((size_t)b * n_split + s) * kH + h];
+        const float l = lse_part[((size_t)b * n_split + s) * n_heads + h];
         const float w = (mx == -INFINITY) ? 0.f : __expf(l - mx);
         coef[tid * kCombineMaxSplits + s] = w;
         total += w;
       }
       const float inv = total > 0.f ? 1.f / total : 0.f;
       for (int s = 0; s < n_split; ++s) coef[tid * kCombineMaxSplits + s] *= inv;
-      if (lse_out) lse_out[(size_t)b * kH + h] = total > 0.f ? mx + __logf(total) : -INFINITY;
+      if (lse_out) lse_out[(size_t)b * n_heads + h] = total > 0.f ? mx + __logf(total) : -INFINITY;
     }
     __syncthreads();
 
@@ -948,7 +953,7 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
         for (int s = 0; s < n_split; ++s) {
           const float a = coef[n * kCombineMaxSplits + s];
           const float4* src =
-              reinterpret_cast<const float4*>(o_f32 + (((size_t)b * n_split + s) * kH + h) * kDl + q * 8);
+              reinterpret_cast<const float4*>(o_f32 + (((size_t)b * n_split + s) * n_heads + h) * kDl + q * 8);
           const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
           acc[0] += a * x0.x; acc[1] += a * x0.y; acc[2] += a * x0.z; acc[3] += a * x0.w;
           acc[4] += a * x1.x; acc[5] += a * x1.y; acc[6] += a * x1.z; acc[7] += a * x1.w;
@@ -990,7 +995,7 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int n = n0 + j;
-        if (n < rows) out[((size_t)(b0 + n) * kH + h) * kDv + e] = __float2bfloat16_rn(__uint_as_float(v[j]));
+        if (n < rows) out[((size_t)(b0 + n) * n_heads + h) * kDv + e] = __float2bfloat16_rn(__uint_as_float(v[j]));
       }
     }
   }

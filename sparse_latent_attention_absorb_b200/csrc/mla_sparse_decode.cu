@@ -11,6 +11,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "dequant.cuh"
 #include "index_check.cuh"
 #include "kernels.cuh"
 #include "mla_sparse_decode.h"
@@ -93,10 +94,11 @@ int get_encoder() {
   return MLA_OK;
 }
 
-// wkv_b as a 2-D bf16 tensor [128*256 rows, 512 columns], boxes of
-// 64 columns x 128 rows, 128-byte swizzle.
-int encode_wkv_b(CUtensorMap* m, const void* wkv_b) {
-  cuuint64_t dims[2] = {(cuuint64_t)kDl, (cuuint64_t)kH * kHeadRows};
+// wkv_b (or a shard of n_heads heads) as a 2-D bf16 tensor
+// [n_heads*256 rows, 512 columns], boxes of 64 columns x 128 rows, 128-byte
+// swizzle.
+int encode_wkv_b(CUtensorMap* m, const void* wkv_b, int n_heads) {
+  cuuint64_t dims[2] = {(cuuint64_t)kDl, (cuuint64_t)n_heads * kHeadRows};
   cuuint64_t strides[1] = {(cuuint64_t)kDl * 2};
   cuuint32_t box[2] = {64, 128};
   cuuint32_t estr[2] = {1, 1};
@@ -106,11 +108,11 @@ int encode_wkv_b(CUtensorMap* m, const void* wkv_b) {
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// q_nope as a 3-D bf16 tensor {d: 128, h: 128, b: B}, boxes of
+// q_nope as a 3-D bf16 tensor {d: 128, h: n_heads, b: B}, boxes of
 // 64 d x 1 head x n_tile rows, 128-byte swizzle (rows past B read as zero).
-int encode_q_nope(CUtensorMap* m, const void* q_nope, int B, int n_tile) {
-  cuuint64_t dims[3] = {(cuuint64_t)kDn, (cuuint64_t)kH, (cuuint64_t)B};
-  cuuint64_t strides[2] = {(cuuint64_t)kDn * 2, (cuuint64_t)kH * kDn * 2};
+int encode_q_nope(CUtensorMap* m, const void* q_nope, int B, int n_tile, int n_heads) {
+  cuuint64_t dims[3] = {(cuuint64_t)kDn, (cuuint64_t)n_heads, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)kDn * 2, (cuuint64_t)n_heads * kDn * 2};
   cuuint32_t box[3] = {64, 1, (cuuint32_t)n_tile};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q_nope), dims, strides, box, estr,
@@ -120,11 +122,11 @@ int encode_q_nope(CUtensorMap* m, const void* q_nope, int B, int n_tile) {
 }
 
 // The mixed latent O~ (single-split rows) as a 3-D bf16 tensor
-// {c: 512, h: 128, b: B}, boxes of 64 c x 1 head x n_tile rows, 128-byte
+// {c: 512, h: n_heads, b: B}, boxes of 64 c x 1 head x n_tile rows, 128-byte
 // swizzle (rows past B read as zero).
-int encode_o_lat(CUtensorMap* m, const void* o_lat, int B, int n_tile) {
-  cuuint64_t dims[3] = {(cuuint64_t)kDl, (cuuint64_t)kH, (cuuint64_t)B};
-  cuuint64_t strides[2] = {(cuuint64_t)kDl * 2, (cuuint64_t)kH * kDl * 2};
+int encode_o_lat(CUtensorMap* m, const void* o_lat, int B, int n_tile, int n_heads) {
+  cuuint64_t dims[3] = {(cuuint64_t)kDl, (cuuint64_t)n_heads, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)kDl * 2, (cuuint64_t)n_heads * kDl * 2};
   cuuint32_t box[3] = {64, 1, (cuuint32_t)n_tile};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(o_lat), dims, strides, box, estr,
@@ -133,11 +135,12 @@ int encode_o_lat(CUtensorMap* m, const void* o_lat, int B, int n_tile) {
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// wo as a 2-D bf16 tensor [dim rows, 16384 columns], boxes of 64 columns x
-// 128 rows, 128-byte swizzle.
-int encode_wo(CUtensorMap* m, const void* wo, int dim) {
-  cuuint64_t dims[2] = {(cuuint64_t)kProjK, (cuuint64_t)dim};
-  cuuint64_t strides[1] = {(cuuint64_t)kProjK * 2};
+// wo (its first k_in columns) as a 2-D bf16 tensor [dim rows, k_in columns]
+// with rows ld elements apart, boxes of 64 columns x 128 rows, 128-byte
+// swizzle.
+int encode_wo(CUtensorMap* m, const void* wo, int dim, int k_in, long long ld) {
+  cuuint64_t dims[2] = {(cuuint64_t)k_in, (cuuint64_t)dim};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
   cuuint32_t box[2] = {(cuuint32_t)kProjKBlock, (cuuint32_t)kProjM};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(wo), dims, strides, box, estr,
@@ -146,13 +149,14 @@ int encode_wo(CUtensorMap* m, const void* wo, int dim) {
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// wo viewed as a 4-D bf16 tensor (64 k, 8 rows of a group, 256 k-blocks,
-// dim/8 groups) with strides (2 B, 32 KB, 128 B, 256 KB): one box {64, 8, 4, 16}
-// is 128 rows x 4 consecutive k-blocks, each row's four 128-byte pieces read
-// back to back, landing as [group][k-block][row][128 B] (128-byte swizzle).
-int encode_wo4(CUtensorMap* m, const void* wo, int dim) {
-  cuuint64_t dims[4] = {(cuuint64_t)kProjKBlock, 8, (cuuint64_t)kProjKBlocks, (cuuint64_t)dim / 8};
-  cuuint64_t strides[3] = {(cuuint64_t)kProjK * 2, (cuuint64_t)kProjKBlock * 2, (cuuint64_t)kProjK * 2 * 8};
+// wo viewed as a 4-D bf16 tensor (64 k, 8 rows of a group, k_in/64 k-blocks,
+// dim/8 groups) with strides (2 B, 2 ld B, 128 B, 16 ld B) (32 KB and 256 KB
+// for the full wo): one box {64, 8, 4, 16} is 128 rows x 4 consecutive
+// k-blocks, each row's four 128-byte pieces read back to back, landing as
+// [group][k-block][row][128 B] (128-byte swizzle).
+int encode_wo4(CUtensorMap* m, const void* wo, int dim, int k_in, long long ld) {
+  cuuint64_t dims[4] = {(cuuint64_t)kProjKBlock, 8, (cuuint64_t)(k_in / kProjKBlock), (cuuint64_t)dim / 8};
+  cuuint64_t strides[3] = {(cuuint64_t)ld * 2, (cuuint64_t)kProjKBlock * 2, (cuuint64_t)ld * 2 * 8};
   cuuint32_t box[4] = {(cuuint32_t)kProjKBlock, 8, (cuuint32_t)kProjKGroupWide, (cuuint32_t)(kProjM / 8)};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(wo), dims, strides, box, estr,
@@ -161,11 +165,11 @@ int encode_wo4(CUtensorMap* m, const void* wo, int dim) {
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// The projection input x as a 2-D bf16 tensor [B rows, 16384 columns], boxes
+// The projection input x as a 2-D bf16 tensor [B rows, k_in columns], boxes
 // of 64 columns x n_tile rows, 128-byte swizzle (rows past B read as zero).
-int encode_proj_x(CUtensorMap* m, const void* x, int B, int n_tile) {
-  cuuint64_t dims[2] = {(cuuint64_t)kProjK, (cuuint64_t)B};
-  cuuint64_t strides[1] = {(cuuint64_t)kProjK * 2};
+int encode_proj_x(CUtensorMap* m, const void* x, int B, int n_tile, int k_in) {
+  cuuint64_t dims[2] = {(cuuint64_t)k_in, (cuuint64_t)B};
+  cuuint64_t strides[1] = {(cuuint64_t)k_in * 2};
   cuuint32_t box[2] = {(cuuint32_t)kProjKBlock, (cuuint32_t)n_tile};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
@@ -207,24 +211,25 @@ bool proj_sizes_ok(int B, int dim) {
 // (f32 partials, then the reduce kernel), otherwise one CTA per tile writes
 // bf16 directly.
 struct ProjPlan {
-  int n_tile = 0, tiles = 0, n_ctas = 0, kgroup = 1;
+  int n_tile = 0, tiles = 0, n_ctas = 0, kgroup = 1, k_blocks = kProjKBlocks;
   bool direct = false;
   size_t partial_bytes = 0;
 };
 
-ProjPlan plan_projection(int B, int dim, int sm_count) {
+ProjPlan plan_projection(int B, int dim, int sm_count, int k_in = kProjK) {
   ProjPlan p;
+  p.k_blocks = k_in / kProjKBlock;
   const int y_tiles = ceil_div(B, kProjNMax);
   p.n_tile = ceil_div(ceil_div(B, y_tiles), 16) * 16;
   p.tiles = y_tiles * (dim / kProjM);
   p.direct = p.tiles >= sm_count;
   // four k-blocks per unit where two such stages fit (split mode only: a
   // direct CTA's tile is 256 units of one k-block)
-  p.kgroup = (!p.direct && p.n_tile <= kProjWideNMax) ? kProjKGroupWide : 1;
+  p.kgroup = (!p.direct && p.n_tile <= kProjWideNMax && p.k_blocks % kProjKGroupWide == 0) ? kProjKGroupWide : 1;
   // split mode: at most one CTA per unit (every CTA owns at least one unit, so
   // the reduce's contributors are exactly the CTAs between a tile's first and
   // last unit) and more CTAs than tiles (a range spans at most two tiles)
-  const long long units = (long long)p.tiles * (kProjKBlocks / p.kgroup);
+  const long long units = (long long)p.tiles * (p.k_blocks / p.kgroup);
   p.n_ctas = p.direct ? p.tiles : (int)(units < sm_count ? units : sm_count);
   p.partial_bytes = p.direct ? 0 : (size_t)2 * p.n_ctas * p.n_tile * kProjM * sizeof(float);
   return p;
@@ -234,15 +239,15 @@ struct WorkspaceLayout {
   size_t q_lat = 0, o_part = 0, lse_part = 0, total = 0;
 };
 
-WorkspaceLayout workspace_layout(int B, int n_split) {
+WorkspaceLayout workspace_layout(int B, int n_split, int n_heads = kH) {
   WorkspaceLayout w;
   size_t off = 0;
   w.q_lat = off;
-  off = round_up(off + (size_t)B * kH * kDl * 2, 256);
+  off = round_up(off + (size_t)B * n_heads * kDl * 2, 256);
   w.o_part = off;  // f32 partials per split, or bf16 O~ when a row is one split
-  off = round_up(off + (size_t)B * n_split * kH * kDl * (n_split == 1 ? 2 : 4), 256);
+  off = round_up(off + (size_t)B * n_split * n_heads * kDl * (n_split == 1 ? 2 : 4), 256);
   w.lse_part = off;
-  off = round_up(off + (size_t)B * n_split * kH * 4, 256);
+  off = round_up(off + (size_t)B * n_split * n_heads * 4, 256);
   w.total = off;
   return w;
 }
@@ -273,44 +278,45 @@ int launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cuda
   return launch_check();
 }
 
-int launch_absorb(const void* q_nope, const void* wkv_b, void* q_lat, int B, int* d_status, cudaStream_t stream) {
+int launch_absorb(const void* q_nope, const void* wkv_b, void* q_lat, int B, int* d_status, cudaStream_t stream,
+                  int n_heads = kH) {
   const int n_tile = B >= kAbsorbNMax ? kAbsorbNMax : ceil_div(B, 16) * 16;
   CUtensorMap tm_w, tm_q;
   int rc;
-  if ((rc = encode_wkv_b(&tm_w, wkv_b)) != MLA_OK) return rc;
-  if ((rc = encode_q_nope(&tm_q, q_nope, B, n_tile)) != MLA_OK) return rc;
-  dim3 grid(kDl / 128, kH, ceil_div(B, kAbsorbNMax));
+  if ((rc = encode_wkv_b(&tm_w, wkv_b, n_heads)) != MLA_OK) return rc;
+  if ((rc = encode_q_nope(&tm_q, q_nope, B, n_tile, n_heads)) != MLA_OK) return rc;
+  dim3 grid(kDl / 128, n_heads, ceil_div(B, kAbsorbNMax));
   return launch_ex(absorb_kernel, grid, dim3(128), absorb_smem_bytes(n_tile), stream, false, tm_w, tm_q,
-                   static_cast<__nv_bfloat16*>(q_lat), B, n_tile, d_status);
+                   static_cast<__nv_bfloat16*>(q_lat), B, n_tile, n_heads, d_status);
 }
 
 int launch_attend(const void* q_lat, const void* q_pe, const void* kv_cache, const void* pe_cache,
                   const int32_t* end_pos, const int32_t* topk_idx, float scale, void* o_part, float* lse_part, int B,
                   int K, int S_max, int n_split, int span, const void* w_next, int* d_status, cudaStream_t stream,
-                  bool pdl, const int32_t* cache_slot = nullptr, int n_slots = 0) {
+                  bool pdl, const int32_t* cache_slot = nullptr, int n_slots = 0, int n_heads = kH) {
   const long long ctas = 2LL * B * n_split;
   if (ctas > 0x7fffffffLL) return MLA_ERR_INVALID_ARG;
   return launch_ex(sparse_attend_kernel, dim3((unsigned)ctas), dim3(kAttendThreads), kAttendSmemBytes, stream, pdl,
                    static_cast<const __nv_bfloat16*>(q_lat), static_cast<const __nv_bfloat16*>(q_pe),
                    static_cast<const __nv_bfloat16*>(kv_cache), static_cast<const __nv_bfloat16*>(pe_cache), end_pos,
                    topk_idx, scale, o_part, lse_part, K, S_max, n_split, span,
-                   static_cast<const __nv_bfloat16*>(w_next), cache_slot, n_slots, d_status);
+                   static_cast<const __nv_bfloat16*>(w_next), cache_slot, n_slots, n_heads, d_status);
 }
 
 int launch_combine(const void* o_part, const float* lse_part, const void* wkv_b, void* out, float* lse_out, int B,
-                   int n_split, int* d_status, cudaStream_t stream, bool pdl) {
+                   int n_split, int* d_status, cudaStream_t stream, bool pdl, int n_heads = kH) {
   const int n_tile = B >= kCombineNMax ? kCombineNMax : ceil_div(B, 16) * 16;
   CUtensorMap tm_w, tm_o;
   int rc;
-  if ((rc = encode_wkv_b(&tm_w, wkv_b)) != MLA_OK) return rc;
+  if ((rc = encode_wkv_b(&tm_w, wkv_b, n_heads)) != MLA_OK) return rc;
   if (n_split == 1) {
-    if ((rc = encode_o_lat(&tm_o, o_part, B, n_tile)) != MLA_OK) return rc;
+    if ((rc = encode_o_lat(&tm_o, o_part, B, n_tile, n_heads)) != MLA_OK) return rc;
   } else {
     tm_o = tm_w;  // unused
   }
-  dim3 grid(kH, ceil_div(B, kCombineNMax));
+  dim3 grid(n_heads, ceil_div(B, kCombineNMax));
   return launch_ex(combine_value_up_kernel, grid, dim3(kCombineThreads), kCombineSmemBytes, stream, pdl, tm_w, tm_o,
-                   o_part, lse_part, static_cast<__nv_bfloat16*>(out), lse_out, B, n_split, n_tile, d_status);
+                   o_part, lse_part, static_cast<__nv_bfloat16*>(out), lse_out, B, n_split, n_tile, n_heads, d_status);
 }
 
 // projection_kernel, then (unless every CTA wrote its tile directly) the
@@ -318,25 +324,26 @@ int launch_combine(const void* o_part, const float* lse_part, const void* wkv_b,
 // projection kernel itself depends programmatically on the kernel before it:
 // it requests its first weight stages before waiting for that kernel.
 int launch_projection(const void* x, const void* wo, void* delta, int B, int dim, const ProjPlan& p, void* partial,
-                      int* d_status, cudaStream_t stream, bool pdl) {
+                      int* d_status, cudaStream_t stream, bool pdl, long long ld_wo = kProjK) {
+  const int k_in = p.k_blocks * kProjKBlock;
   CUtensorMap tm_wo, tm_wo4, tm_x;
   int rc;
-  if ((rc = encode_wo(&tm_wo, wo, dim)) != MLA_OK) return rc;
+  if ((rc = encode_wo(&tm_wo, wo, dim, k_in, ld_wo)) != MLA_OK) return rc;
   if (p.kgroup == 1)
     tm_wo4 = tm_wo;  // unused
-  else if ((rc = encode_wo4(&tm_wo4, wo, dim)) != MLA_OK)
+  else if ((rc = encode_wo4(&tm_wo4, wo, dim, k_in, ld_wo)) != MLA_OK)
     return rc;
-  if ((rc = encode_proj_x(&tm_x, x, B, p.n_tile)) != MLA_OK) return rc;
+  if ((rc = encode_proj_x(&tm_x, x, B, p.n_tile, k_in)) != MLA_OK) return rc;
   if ((rc = launch_ex(projection_kernel, dim3((unsigned)p.n_ctas), dim3(kProjThreads),
                       proj_smem_bytes(p.n_tile, p.kgroup), stream, pdl, tm_wo, tm_wo4, tm_x,
                       static_cast<float*>(partial), static_cast<__nv_bfloat16*>(delta), B, dim, p.n_tile, p.n_ctas,
-                      p.direct ? 1 : 0, p.kgroup, d_status)) != MLA_OK)
+                      p.direct ? 1 : 0, p.kgroup, p.k_blocks, d_status)) != MLA_OK)
     return rc;
   if (p.direct) return MLA_OK;
   dim3 grid((unsigned)p.tiles, ceil_div(p.n_tile, kProjReduceRows));
   return launch_ex(projection_reduce_kernel, grid, dim3(kProjReduceThreads), 0, stream, true,
                    static_cast<const float*>(partial), static_cast<__nv_bfloat16*>(delta), B, dim, p.n_tile,
-                   p.n_ctas, p.kgroup);
+                   p.n_ctas, p.kgroup, p.k_blocks);
 }
 
 int prepare(DeviceInfo** info) {
@@ -459,7 +466,7 @@ namespace {
 int run_rows(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
              const int32_t* end_pos, const int32_t* topk_idx, const void* wkv_b, float scale, void* out, int B, int K,
              int S_max, const int32_t* cache_slot, int n_slots, void* workspace, size_t workspace_bytes,
-             float* lse_out, int* d_status, cudaStream_t stream) {
+             float* lse_out, int* d_status, cudaStream_t stream, int n_heads = kH) {
   const void* ptrs[] = {q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, out};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return MLA_ERR_INVALID_ARG;
@@ -471,7 +478,7 @@ int run_rows(const void* q_nope, const void* q_pe, const void* kv_cache, const v
   if (rc != MLA_OK) return rc;
   int n_split = 0, span = 0;
   plan_splits(B, K, info->sm_count, &n_split, &span);
-  const WorkspaceLayout wl = workspace_layout(B, n_split);
+  const WorkspaceLayout wl = workspace_layout(B, n_split, n_heads);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < wl.total)
     return MLA_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -487,13 +494,13 @@ int run_rows(const void* q_nope, const void* q_pe, const void* kv_cache, const v
   // only where it reads that kernel's output.  The absorption kernel is an
   // ordinary launch, so all earlier work in the stream (whatever wrote the
   // caches and indices) has finished before any of the three starts.
-  if ((rc = launch_absorb(q_nope, wkv_b, q_lat, B, d_status, stream)) != MLA_OK) return rc;
+  if ((rc = launch_absorb(q_nope, wkv_b, q_lat, B, d_status, stream, n_heads)) != MLA_OK) return rc;
   // The attention kernel also pulls W_UV into L2 near its end, for the
   // value-up kernel.
   if ((rc = launch_attend(q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, scale, o_part, lse_part, B, K, S_max,
-                          n_split, span, wkv_b, d_status, stream, true, cache_slot, n_slots)) != MLA_OK)
+                          n_split, span, wkv_b, d_status, stream, true, cache_slot, n_slots, n_heads)) != MLA_OK)
     return rc;
-  return launch_combine(o_part, lse_part, wkv_b, out, lse_out, B, n_split, d_status, stream, true);
+  return launch_combine(o_part, lse_part, wkv_b, out, lse_out, B, n_split, d_status, stream, true, n_heads);
 }
 }  // namespace
 
@@ -515,6 +522,40 @@ extern "C" int mla_sparse_prefill(const void* q_nope, const void* q_pe, const vo
   if (!cache_slot || !aligned16(cache_slot) || n_slots < 1) return MLA_ERR_INVALID_ARG;
   return run_rows(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, scale, out, R, K, S_max, cache_slot,
                   n_slots, workspace, workspace_bytes, lse_out, d_status, stream);
+}
+
+// One tensor-parallel shard of the decode (see the header): the same three
+// kernels over n_heads consecutive heads.
+extern "C" size_t mla_sparse_decode_heads_workspace_size(int B, int K, int S_max, int n_heads) {
+  if (!sizes_ok(B, K, S_max) || n_heads < 1 || n_heads > kH) return 0;
+  int n_split = 0, span = 0;
+  plan_splits(B, K, planning_sm_count(), &n_split, &span);
+  return workspace_layout(B, n_split, n_heads).total;
+}
+
+extern "C" int mla_sparse_decode_heads(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                                       const int32_t* end_pos, const int32_t* topk_idx, const void* wkv_b,
+                                       float scale, void* out, int B, int K, int S_max, int n_heads, void* workspace,
+                                       size_t workspace_bytes, float* lse_out, int* d_status, cudaStream_t stream) {
+  if (n_heads < 1 || n_heads > kH) return MLA_ERR_INVALID_ARG;
+  return run_rows(q_nope, q_pe, kv_cache, pe_cache, end_pos, topk_idx, wkv_b, scale, out, B, K, S_max, nullptr, B,
+                  workspace, workspace_bytes, lse_out, d_status, stream, n_heads);
+}
+
+// fp8 block dequantisation (see the header).
+extern "C" int mla_dequant_fp8_blocks(const void* w_fp8, const float* scale, void* w_bf16, int rows, int cols,
+                                      cudaStream_t stream) {
+  if (!w_fp8 || !scale || !w_bf16 || !aligned16(w_fp8) || !aligned16(w_bf16)) return MLA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(scale) & 3u) return MLA_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 16 || cols % 16 || (long long)rows * cols > (1LL << 40)) return MLA_ERR_INVALID_ARG;
+  DeviceInfo* info = nullptr;
+  int rc = prepare(&info);
+  if (rc != MLA_OK) return rc;
+  const long long n_vec = (long long)rows * (cols / 16);
+  long long blocks = (n_vec + kDequantThreads - 1) / kDequantThreads;
+  if (blocks > 8LL * info->sm_count) blocks = 8LL * info->sm_count;
+  return launch_ex(dequant_fp8_blocks_kernel, dim3((unsigned)blocks), dim3(kDequantThreads), 0, stream, false,
+                   static_cast<const uint8_t*>(w_fp8), scale, static_cast<__nv_bfloat16*>(w_bf16), rows, cols);
 }
 
 // Index validation (see the header): repeated valid entries of a row.
@@ -678,6 +719,33 @@ extern "C" int mla_output_projection(const void* x, const void* wo, void* delta,
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
     return MLA_ERR_WORKSPACE;
   return launch_projection(x, wo, delta, B, dim, p, workspace, d_status, stream, false);
+}
+
+// The projection of a tensor-parallel shard (see the header): x [B, k_in],
+// wo's rows ld_wo elements apart, its first k_in columns used.
+extern "C" size_t mla_output_projection_shard_workspace_size(int B, int dim, int k_in) {
+  if (!proj_sizes_ok(B, dim) || k_in < kProjKBlock || k_in > kProjK || k_in % kProjKBlock) return 0;
+  const ProjPlan p = plan_projection(B, dim, planning_sm_count(), k_in);
+  return p.partial_bytes > 0 ? p.partial_bytes : 256;
+}
+
+extern "C" int mla_output_projection_shard(const void* x, const void* wo, long long ld_wo, void* delta, int B,
+                                           int dim, int k_in, void* workspace, size_t workspace_bytes, int* d_status,
+                                           cudaStream_t stream) {
+  const void* ptrs[] = {x, wo, delta};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (!proj_sizes_ok(B, dim) || k_in < kProjKBlock || k_in > kProjK || k_in % kProjKBlock) return MLA_ERR_INVALID_ARG;
+  if (ld_wo < k_in || ld_wo % 8 || ld_wo > (1LL << 31)) return MLA_ERR_INVALID_ARG;  // rows 16-byte aligned
+  DeviceInfo* info = nullptr;
+  int rc = prepare(&info);
+  if (rc != MLA_OK) return rc;
+  const ProjPlan p = plan_projection(B, dim, info->sm_count, k_in);
+  const size_t need = p.partial_bytes > 0 ? p.partial_bytes : 256;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+    return MLA_ERR_WORKSPACE;
+  return launch_projection(x, wo, delta, B, dim, p, workspace, d_status, stream, false, ld_wo);
 }
 
 // The decode step followed by the output projection: the workspace holds the

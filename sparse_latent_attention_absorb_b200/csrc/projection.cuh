@@ -6,7 +6,10 @@
 //   delta[b, n] = bf16( sum_k x[b, k] * wo[n, k] ),   k < 16384, n < dim
 //
 // wo is the torch Linear weight [dim, 16384] (k contiguous); the pages show no
-// bias.  At decode sizes the projection is a stream over wo (235 MB at
+// bias.  The kernels take the input width as a runtime multiple of 64 and wo
+// with a row stride, so a tensor-parallel shard projects its own heads'
+// outputs through its column slice of wo (the row-parallel partial, summed
+// over the shards afterwards).  At decode sizes the projection is a stream over wo (235 MB at
 // dim = 7168) with a narrow batch, so it is written as a weight stream:
 //
 //   projection_kernel  persistent swap-AB tcgen05 GEMM.  An output tile is
@@ -36,9 +39,9 @@
 
 namespace mla {
 
-constexpr int kProjK = kH * kDv;                   // 16384 inputs per row
+constexpr int kProjK = kH * kDv;                   // 16384 inputs per row (all heads)
 constexpr int kProjKBlock = 64;                    // k per unit: one 128-byte swizzle row
-constexpr int kProjKBlocks = kProjK / kProjKBlock; // 256 units per row tile
+constexpr int kProjKBlocks = kProjK / kProjKBlock; // 256 k-blocks per row tile (all heads)
 constexpr int kProjM = 128;                        // wo rows per tile (MMA M)
 constexpr int kProjNMax = 256;                     // batch rows per tile (MMA N, TMA box)
 constexpr int kProjStagesMax = 8;
@@ -80,14 +83,14 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_wo4,
                   const __grid_constant__ CUtensorMap tm_x, float* __restrict__ partial,
                   __nv_bfloat16* __restrict__ delta, int B, int dim, int n_tile, int n_ctas, int direct, int kgroup,
-                  int* d_status) {
+                  int k_blocks, int* d_status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
   const int stages = proj_stages(n_tile, kgroup);
   const int stage_bytes = proj_stage_bytes(n_tile, kgroup);
-  const int upt = kProjKBlocks / kgroup;        // units per tile
+  const int upt = k_blocks / kgroup;            // units per tile
   const int a_bytes = kgroup * kProjABytes;     // wo part of a stage; the x boxes follow
   const int m_tiles = dim / kProjM;
   const long long U = (long long)m_tiles * ((B + n_tile - 1) / n_tile) * upt;
@@ -257,14 +260,14 @@ constexpr int kProjReduceThreads = kProjReduceRows * 32;
 
 __global__ void __launch_bounds__(kProjReduceThreads)
 projection_reduce_kernel(const float* __restrict__ partial, __nv_bfloat16* __restrict__ delta, int B, int dim,
-                         int n_tile, int n_ctas, int kgroup) {
+                         int n_tile, int n_ctas, int kgroup, int k_blocks) {
   const int t = blockIdx.x;
   const int m_tiles = dim / kProjM;
   const int m = t % m_tiles;
   const int row0 = (t / m_tiles) * n_tile;
   const int j = blockIdx.y * kProjReduceRows + (int)(threadIdx.x >> 5);  // row within the tile
   const int n4 = (int)(threadIdx.x & 31) * 4;
-  const int upt = kProjKBlocks / kgroup;  // units per tile
+  const int upt = k_blocks / kgroup;  // units per tile
   const int U = m_tiles * ((B + n_tile - 1) / n_tile) * upt;
   int c_lo, c_hi;  // the CTAs holding the tile's units
   proj_tile_ctas<int>(t, upt, U, n_ctas, &c_lo, &c_hi);

@@ -233,3 +233,21 @@ def generate_prefill(B: int, seqlen: int, K: int, seed: int = 2101) -> dict:
         "scale": SCALE,
         "B": B, "seqlen": seqlen,
     }
+
+
+def generate_fp8_wkv_b(n_heads: int = H, seed: int = 2201) -> dict:
+    """wkv_b in the fp8 block format the decode excerpt can find it in
+    (``wkv_b.weight`` with ``wkv_b.scale``), on the CPU: codes uint8
+    [n_heads*256, 512] (OCP E4M3) and scale f32 [n_heads*2, 4], one per
+    128 x 128 block.  Drawn as bf16-distributed weights N(0, 512^-0.5), each
+    block scaled so that its largest magnitude maps to 448 (the largest E4M3
+    value) and converted by torch's float8_e4m3fn cast."""
+    gen = torch.Generator().manual_seed(seed)
+    rows, cols = n_heads * (D_NOPE + D_V), D_LAT
+    w = torch.randn((rows, cols), generator=gen, dtype=torch.float32) * D_LAT ** -0.5
+    blocks = w.view(rows // 128, 128, cols // 128, 128)
+    amax = blocks.abs().amax(dim=(1, 3)).clamp_min(1e-12)
+    scale = (amax / 448.0).to(torch.float32)
+    q = (blocks / scale[:, None, :, None]).view(rows, cols)
+    codes = q.to(torch.float8_e4m3fn).view(torch.uint8)
+    return {"codes": codes.contiguous(), "scale": scale.contiguous()}

@@ -227,3 +227,54 @@ def test_index_check_flag_is_a_process_wide_switch(lib):
         assert lib.mla_set_index_checks(0) == 0
     finally:
         lib.mla_set_index_checks(prev)
+
+
+def test_shard_entry_points_reject_bad_arguments_without_a_launch(lib):
+    A = 0x10000
+    p7 = [_fake(A)] * 7
+
+    def dec(n_heads=64, B=2, K=16, S=32, ptrs=None, ws=_fake(A)):
+        p = ptrs or p7
+        return lib.mla_sparse_decode_heads(*p[:7], ctypes.c_float(0.07), _fake(A), B, K, S, n_heads, ws, 1 << 30,
+                                           None, None, None)
+
+    for n in (0, -1, 129):
+        assert dec(n_heads=n) == INVALID_ARG
+    for i in range(7):
+        bad = list(p7)
+        bad[i] = _fake(A + 4)
+        assert dec(ptrs=bad) == INVALID_ARG
+    assert lib.mla_sparse_decode_heads_workspace_size(2, 16, 32, 0) == 0
+    assert lib.mla_sparse_decode_heads_workspace_size(2, 16, 32, 129) == 0
+    # a shard's scratch scales with its heads; all 128 heads = the decode's
+    assert lib.mla_sparse_decode_heads_workspace_size(64, 2048, 4096, 128) == \
+        lib.mla_sparse_decode_workspace_size(64, 2048, 4096)
+    assert lib.mla_sparse_decode_heads_workspace_size(64, 2048, 4096, 64) < \
+        lib.mla_sparse_decode_workspace_size(64, 2048, 4096)
+
+    def proj(k_in=8192, ld=16384, dim=7168, B=4, x=_fake(A), wo=_fake(A)):
+        return lib.mla_output_projection_shard(x, wo, ld, _fake(A), B, dim, k_in, _fake(A), 1 << 30, None, None)
+
+    for k_in in (0, 32, 100, 16384 + 64):
+        assert proj(k_in=k_in) == INVALID_ARG
+    for ld in (8191, 8196, 1 << 32):  # shorter than k_in, rows not 16-byte aligned, too long
+        assert proj(ld=ld) == INVALID_ARG
+    assert proj(dim=100) == INVALID_ARG
+    assert proj(x=_fake(A + 8)) == INVALID_ARG
+    assert lib.mla_output_projection_shard_workspace_size(4, 7168, 100) == 0
+    assert lib.mla_output_projection_shard_workspace_size(4, 7168, 16384) == \
+        lib.mla_output_projection_workspace_size(4, 7168)
+
+
+def test_dequant_rejects_bad_arguments_without_a_launch(lib):
+    A = 0x10000
+
+    def call(w=_fake(A), s=_fake(A), o=_fake(A), rows=256, cols=512):
+        return lib.mla_dequant_fp8_blocks(w, s, o, rows, cols, None)
+
+    assert call(w=None) == INVALID_ARG
+    assert call(o=_fake(A + 8)) == INVALID_ARG
+    assert call(s=_fake(A + 2)) == INVALID_ARG
+    assert call(rows=0) == INVALID_ARG
+    assert call(cols=8) == INVALID_ARG
+    assert call(cols=520 + 4) == INVALID_ARG
