@@ -239,12 +239,21 @@ int mla_sparse_decode_noalloc(const void* q_nope, const void* q_pe, const void* 
  *   workspace / workspace_bytes: device scratch, 256-byte aligned, at least
  *            mla_sparse_decode_host_workspace_size(B, K, S_max) bytes: the
  *            decode's scratch plus device copies of the four inputs and out
- * Enqueues on `stream`, in order: one cudaMemcpyAsync per input, the decode
- * step, one cudaMemcpyAsync of out to h_out.  h_out is complete once `stream`
- * has passed this point; the host buffers must stay valid until then.
- * Consecutive calls overlap when they alternate between streams, each with
- * its own workspace.  Returns an mla_status.
+ * Enqueues on `stream`, in order: the uploads, the decode step, one
+ * cudaMemcpyAsync of out to h_out.  The uploads are one cudaMemcpyAsync per
+ * input, or a single one when the four inputs sit in one host buffer at the
+ * offsets mla_sparse_decode_host_input_layout gives (the staging area's own
+ * layout: fewer, larger copies run closer to the link's bandwidth).  h_out
+ * is complete once `stream` has passed this point; the host buffers must stay
+ * valid until then.  Consecutive calls overlap when they rotate between
+ * streams, each with its own workspace.  Returns an mla_status.
+ *
+ * mla_sparse_decode_host_input_layout: byte offsets of h_q_nope, h_q_pe,
+ * h_end_pos and h_topk_idx (offsets[0..3], offsets[0] = 0) in such a packed
+ * host buffer, and its size as the return value (0 for invalid sizes);
+ * offsets may be NULL.
  */
+size_t mla_sparse_decode_host_input_layout(int B, int K, int S_max, size_t* offsets);
 size_t mla_sparse_decode_host_workspace_size(int B, int K, int S_max);
 int mla_sparse_decode_host(const void* h_q_nope, const void* h_q_pe, const int32_t* h_end_pos,
                            const int32_t* h_topk_idx, const void* kv_cache, const void* pe_cache, const void* wkv_b,

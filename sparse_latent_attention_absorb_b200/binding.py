@@ -24,7 +24,7 @@ STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_WORKSPACE", 3: "MLA
 # Every symbol the public header declares.
 EXPORTS = ("mla_status_string", "mla_num_splits", "mla_sparse_decode_workspace_size", "mla_sparse_decode",
            "mla_absorb_q", "mla_sparse_attend", "mla_combine_value_up", "mla_sparse_decode_noalloc",
-           "mla_sparse_decode_host_workspace_size", "mla_sparse_decode_host",
+           "mla_sparse_decode_host_workspace_size", "mla_sparse_decode_host", "mla_sparse_decode_host_input_layout",
            "mla_output_projection_workspace_size", "mla_output_projection",
            "mla_sparse_decode_project_workspace_size", "mla_sparse_decode_project", "mla_sparse_prefill",
            "mla_selftest_wait_timeout", "mla_check_topk_indices", "mla_set_index_checks",
@@ -68,6 +68,8 @@ def load_library():
     lib.mla_sparse_decode_noalloc.argtypes = [p, p, p, p, p, p, p, f, p, i, i, i, p, p, p]
     lib.mla_sparse_decode_host_workspace_size.restype = sz
     lib.mla_sparse_decode_host_workspace_size.argtypes = [i, i, i]
+    lib.mla_sparse_decode_host_input_layout.restype = sz
+    lib.mla_sparse_decode_host_input_layout.argtypes = [i, i, i, p]
     lib.mla_sparse_decode_host.restype = i
     lib.mla_sparse_decode_host.argtypes = [p, p, p, p, p, p, p, f, p, i, i, i, p, sz, p, p, p]
     lib.mla_output_projection_workspace_size.restype = sz
@@ -550,3 +552,27 @@ class Fp8Wkvb:
         if self._bf16 is None:
             self._bf16 = mla_dequant_fp8_blocks(self.w_fp8, self.scale, stream=stream)
         return self._bf16
+
+
+def host_input_buffer(B: int, K: int, S_max: int):
+    """A pinned host buffer laid out like the host entry point's staging area,
+    and views of its four inputs (q_nope, q_pe, end_pos, topk_idx): filling
+    the views and passing them to mla_sparse_decode_host uploads them in one
+    copy."""
+    lib = load_library()
+    offs = (ctypes.c_size_t * 4)()
+    total = lib.mla_sparse_decode_host_input_layout(B, K, S_max, offs)
+    if total == 0:
+        raise MLAError(1, "mla_sparse_decode_host_input_layout")
+    buf = torch.empty(total, dtype=torch.uint8).pin_memory()
+
+    def view(off, dtype, shape):
+        n = 1
+        for d_ in shape:
+            n *= d_
+        return buf[off:off + n * torch.tensor([], dtype=dtype).element_size()].view(dtype).view(shape)
+
+    return buf, {"q_nope": view(offs[0], torch.bfloat16, (B, H, D_NOPE)),
+                 "q_pe": view(offs[1], torch.bfloat16, (B, H, D_ROPE)),
+                 "end_pos": view(offs[2], torch.int32, (B,)),
+                 "topk_idx": view(offs[3], torch.int32, (B, K))}

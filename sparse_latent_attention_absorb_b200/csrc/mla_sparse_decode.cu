@@ -648,6 +648,20 @@ HostStaging host_staging(int B, int K, int n_split) {
 }
 }  // namespace
 
+extern "C" size_t mla_sparse_decode_host_input_layout(int B, int K, int S_max, size_t* offsets) {
+  if (!sizes_ok(B, K, S_max)) return 0;
+  int n_split = 0, span = 0;
+  plan_splits(B, K, planning_sm_count(), &n_split, &span);
+  const HostStaging hs = host_staging(B, K, n_split);
+  if (offsets) {
+    offsets[0] = 0;
+    offsets[1] = hs.q_pe - hs.q_nope;
+    offsets[2] = hs.end_pos - hs.q_nope;
+    offsets[3] = hs.topk_idx - hs.q_nope;
+  }
+  return hs.topk_idx + (size_t)B * K * 4 - hs.q_nope;
+}
+
 extern "C" size_t mla_sparse_decode_host_workspace_size(int B, int K, int S_max) {
   if (!sizes_ok(B, K, S_max)) return 0;
   int n_split = 0, span = 0;
@@ -680,13 +694,25 @@ extern "C" int mla_sparse_decode_host(const void* h_q_nope, const void* h_q_pe, 
   int32_t* d_end_pos = reinterpret_cast<int32_t*>(ws + hs.end_pos);
   int32_t* d_topk_idx = reinterpret_cast<int32_t*>(ws + hs.topk_idx);
   void* d_out = ws + hs.out;
-  // one plain asynchronous copy per tensor (pinned host memory makes them
-  // truly asynchronous; pageable memory works but stages through the driver)
-  if (cudaMemcpyAsync(d_q_nope, h_q_nope, (size_t)B * kH * kDn * 2, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-      cudaMemcpyAsync(d_q_pe, h_q_pe, (size_t)B * kH * kDr * 2, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-      cudaMemcpyAsync(d_end_pos, h_end_pos, (size_t)B * 4, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-      cudaMemcpyAsync(d_topk_idx, h_topk_idx, (size_t)B * K * 4, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+  // Host inputs laid out like the staging area (one buffer, the offsets of
+  // mla_sparse_decode_host_input_layout) go up in a single copy; otherwise one
+  // plain asynchronous copy per tensor.  Pinned host memory makes them truly
+  // asynchronous; pageable memory works but stages through the driver.
+  const char* h0 = static_cast<const char*>(h_q_nope);
+  const bool packed = static_cast<const char*>(h_q_pe) == h0 + (hs.q_pe - hs.q_nope) &&
+                      reinterpret_cast<const char*>(h_end_pos) == h0 + (hs.end_pos - hs.q_nope) &&
+                      reinterpret_cast<const char*>(h_topk_idx) == h0 + (hs.topk_idx - hs.q_nope);
+  if (packed) {
+    if (cudaMemcpyAsync(d_q_nope, h_q_nope, hs.topk_idx + (size_t)B * K * 4 - hs.q_nope, cudaMemcpyHostToDevice,
+                        stream) != cudaSuccess)
+      return MLA_ERR_CUDA;
+  } else if (cudaMemcpyAsync(d_q_nope, h_q_nope, (size_t)B * kH * kDn * 2, cudaMemcpyHostToDevice, stream) !=
+                 cudaSuccess ||
+             cudaMemcpyAsync(d_q_pe, h_q_pe, (size_t)B * kH * kDr * 2, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+             cudaMemcpyAsync(d_end_pos, h_end_pos, (size_t)B * 4, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+             cudaMemcpyAsync(d_topk_idx, h_topk_idx, (size_t)B * K * 4, cudaMemcpyHostToDevice, stream) != cudaSuccess) {
     return MLA_ERR_CUDA;
+  }
   rc = mla_sparse_decode(d_q_nope, d_q_pe, kv_cache, pe_cache, d_end_pos, d_topk_idx, wkv_b, scale, d_out, B, K,
                          S_max, ws, hs.q_nope, lse_out, d_status, stream);
   if (rc != MLA_OK) return rc;

@@ -78,3 +78,38 @@ def test_host_entry_on_two_alternating_streams():
         ref = pkg.mla_sparse_decode(s_["q_nope"].to(DEV), s_["q_pe"].to(DEV), kv, pe, s_["end_pos"].to(DEV),
                                     s_["topk_idx"].to(DEV), ws_w[i], s_["scale"])
         assert torch.equal(outs[i].view(torch.int16), ref.cpu().view(torch.int16))
+
+
+def test_packed_input_layout_matches_the_staging_offsets():
+    lib = binding.load_library()
+    for B, K, S in ((1, 256, 1001), (64, 2048, 32768), (7, 100, 300)):
+        offs = (ctypes.c_size_t * 4)()
+        total = lib.mla_sparse_decode_host_input_layout(B, K, S, offs)
+        sizes = [B * 128 * 128 * 2, B * 128 * 64 * 2, B * 4, B * K * 4]
+        assert offs[0] == 0
+        for i in range(3):  # each tensor follows the previous one, 256-byte aligned
+            assert offs[i + 1] == -(-(offs[i] + sizes[i]) // 256) * 256
+        assert total == offs[3] + sizes[3]
+    assert lib.mla_sparse_decode_host_input_layout(0, 1, 1, None) == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["small_b80_ctx700_top300", "small_b2_ctx300_top100"])
+def test_packed_host_inputs_match_separate_ones(name):
+    d = wl.generate(name)
+    B, K, S = d["q_nope"].shape[0], d["topk_idx"].shape[1], d["kv_cache"].shape[1]
+    kv, pe, w = d["kv_cache"].to(DEV), d["pe_cache"].to(DEV), d["wkv_b"].to(DEV)
+    buf, views = binding.host_input_buffer(B, K, S)
+    for k, v in views.items():
+        v.copy_(d[k])
+    ws = torch.empty(pkg.host_workspace_size(B, K, S), dtype=torch.uint8, device=DEV)
+    out_packed = torch.empty((B, 128, 128), dtype=torch.bfloat16).pin_memory()
+    pkg.mla_sparse_decode_host(views["q_nope"], views["q_pe"], views["end_pos"], views["topk_idx"], kv, pe, w,
+                               d["scale"], out_packed, ws)
+    torch.cuda.synchronize()
+    hin = {k: _pinned(d[k]) for k in ("q_nope", "q_pe", "end_pos", "topk_idx")}
+    out_sep = torch.empty((B, 128, 128), dtype=torch.bfloat16).pin_memory()
+    pkg.mla_sparse_decode_host(hin["q_nope"], hin["q_pe"], hin["end_pos"], hin["topk_idx"], kv, pe, w, d["scale"],
+                               out_sep, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out_packed.view(torch.int16), out_sep.view(torch.int16))
