@@ -53,6 +53,32 @@ constexpr int kAbsorbSmemA = 2 * 64 * 128 * 2;                      // 32 KB
 __host__ __device__ constexpr int absorb_smem_bytes(int n) { return kAbsorbSmemA + 2 * n * 128 + 256 + kSmemAlignPad; }
 constexpr int kAbsorbSmemBytes = absorb_smem_bytes(kAbsorbNMax);
 
+// Whole-kernel stamps of the trace build (globaltimer ns; earliest start via
+// atomicMin, latest end via atomicMax), reset by mla_trace_reset().
+enum KernelEvent {
+  kKeAbsorbStart = 0,  // min over CTAs
+  kKeAbsorbEnd,        // max over CTAs
+  kKeCombineStart,     // min over CTAs
+  kKeCombineWaited,    // max over CTAs: past the wait on the attention kernel
+  kKeCombineEnd,       // max over CTAs
+  kKeCombineFirstWaited,  // min over CTAs: past the wait on the attention kernel
+  kKeCombineIssued,    // max over CTAs: every k-block landed and its MMAs issued
+  kKeCombineMmaDone,   // max over CTAs: accumulator complete
+  kKernelEvents
+};
+#ifdef MLA_TRACE
+__device__ unsigned long long g_mla_kernel_ns[kKernelEvents];
+#define MLA_KERNEL_STAMP_MIN(ev) atomicMin(&g_mla_kernel_ns[(ev)], (unsigned long long)global_timer_ns())
+#define MLA_KERNEL_STAMP_MAX(ev) atomicMax(&g_mla_kernel_ns[(ev)], (unsigned long long)global_timer_ns())
+#else
+#define MLA_KERNEL_STAMP_MIN(ev) \
+  do {                           \
+  } while (0)
+#define MLA_KERNEL_STAMP_MAX(ev) \
+  do {                           \
+  } while (0)
+#endif
+
 __global__ void __launch_bounds__(128, 1)
 absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
               __nv_bfloat16* __restrict__ q_lat, int B, int n_tile, int n_heads, int* d_status) {
@@ -75,6 +101,7 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
   const uint32_t tmem_cols = n_tile <= 32 ? 32u : (n_tile <= 64 ? 64u : 128u);
   // The loads go out first (TMA needs no TMEM); TMEM is allocated meanwhile.
   if (tid == 0) {
+    MLA_KERNEL_STAMP_MIN(kKeAbsorbStart);
     *abort_flag = 0;
     mbar_init(bar_load, 1);
     mbar_init(bar_mma, 1);
@@ -131,6 +158,7 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, tmem_cols);
+  if (tid == 0) MLA_KERNEL_STAMP_MAX(kKeAbsorbEnd);
 }
 
 // =============================================================================
@@ -295,17 +323,38 @@ enum TraceEvent {
   kTrEvents
 };
 constexpr int kTraceTiles = 512;
+// Per-cluster milestones of the trace build (globaltimer ns, CTA rank 0 of
+// every cluster), read back with mla_trace_cluster_fetch().
+enum ClusterEvent {
+  kCeStart = 0,    // barriers and TMEM ready (after the cluster barrier)
+  kCeQuery,        // MMA thread: query half in TMEM
+  kCeFirstTile,    // MMA thread: first tile's rows landed
+  kCeLastQk,       // MMA thread: last QK issued
+  kCeLastPv,       // PV thread: last PV issued
+  kCePvDone,       // softmax: last PV complete (epilogue may read O)
+  kCeEnd,          // every thread past the epilogue
+  kCeClocks,       // SM clock cycles from kCeStart to kCeEnd (clock64)
+  kClusterEvents
+};
+constexpr int kTraceClusters = 4096;
 #ifdef MLA_TRACE
 __device__ long long g_mla_trace[2 * kTrEvents * kTraceTiles];
-__device__ unsigned long long g_mla_cluster_ns[2 * 4096];  // per cluster: start, end (globaltimer)
+__device__ unsigned long long g_mla_cluster_ns[kClusterEvents * kTraceClusters];
 #define MLA_TRACE_STAMP(ev, tile)                                                               \
   do {                                                                                           \
     if ((blockIdx.x >> 1) == 0 && (tile) < kTraceTiles)                                          \
       g_mla_trace[(rank * kTrEvents + (ev)) * kTraceTiles + (tile)] = clock64();                 \
   } while (0)
+#define MLA_CLUSTER_STAMP(ev)                                                                    \
+  do {                                                                                           \
+    if (rank == 0 && unit < kTraceClusters) g_mla_cluster_ns[unit * kClusterEvents + (ev)] = global_timer_ns(); \
+  } while (0)
 #else
 #define MLA_TRACE_STAMP(ev, tile) \
   do {                            \
+  } while (0)
+#define MLA_CLUSTER_STAMP(ev) \
+  do {                        \
   } while (0)
 #endif
 
@@ -381,7 +430,8 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
   const uint32_t tmem = bars->tmem_addr;
   grid_dep_launch();  // the combine kernel may start loading its weights
 #ifdef MLA_TRACE
-  if (rank == 0 && tid == 0 && unit < 4096) g_mla_cluster_ns[2 * unit] = global_timer_ns();
+  const long long clk_start = clock64();
+  if (tid == 0) MLA_CLUSTER_STAMP(kCeStart);
 #endif
 
   if (warp >= kGatherWarp0) {
@@ -489,8 +539,10 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       const uint64_t d_pe = smem_desc_sw64(sStage + 4 * kLatBlock, 512);    // QK B, rotary, K-major
       const uint64_t d_qpe = smem_desc_sw64(sQpe, 512);                     // QK A, rotary, K-major
       wait(smem_u32(&bars->q_full), 0, ab);
+      MLA_CLUSTER_STAMP(kCeQuery);
       for (int qk = 0, st = 0; qk < n_tiles; ++qk, st = (st + 1 == kStages) ? 0 : st + 1) {
         wait(smem_u32(&bars->kv_full[st]), (qk / kStages) & 1, ab);
+        if (qk == 0) MLA_CLUSTER_STAMP(kCeFirstTile);
         MLA_TRACE_STAMP(kTrQkKv, qk);
         if (qk > 0) wait(smem_u32(&bars->s_empty), (qk - 1) & 1, ab);
         MLA_TRACE_STAMP(kTrQkWoke, qk);
@@ -510,6 +562,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
         *reinterpret_cast<volatile int*>(&bars->qk_issued) = qk + 1;
         MLA_TRACE_STAMP(kTrQkIssued, qk);
       }
+      MLA_CLUSTER_STAMP(kCeLastQk);
     }
     __syncwarp();
   } else if (warp == kPvWarp) {
@@ -537,6 +590,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
         mma_commit(smem_u32(&bars->p_free[pv & 1]));
         MLA_TRACE_STAMP(kTrPvIssued, pv);
       }
+      MLA_CLUSTER_STAMP(kCeLastPv);
     }
     __syncwarp();
   } else {
@@ -788,11 +842,17 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       // the last PV done implies every MMA of the split is done
       wait(smem_u32(&bars->p_free[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, ab);
       tc_fence_after();
+      if (leader && grp == 0) MLA_CLUSTER_STAMP(kCePvDone);
     }
     const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
     // A row of one split is final here: its mixed latent O~ goes out in bf16
     // (the value-up operand); several splits keep f32 partials for the merge.
+    // The ring is idle once the last PV is done, so each thread stages its
+    // 128-column half row there (rows padded by 16 bytes: the 32 rows of a
+    // warp fall on distinct banks) and writes it out with one bulk copy.
     const size_t orow = (((size_t)b * n_split + split) * n_heads + (live ? i : 0)) * kDl + rank * 256 + 128 * grp;
+    const uint32_t row_bytes = n_split == 1 ? 128u * 2u : 128u * 4u;
+    const uint32_t stg = sStage + (uint32_t)(grp * kH + i) * (row_bytes + 16u);
 #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {
       uint32_t ov[32];
@@ -803,27 +863,32 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
 #pragma unroll
         for (int t = 0; t < 32; ++t) ov[t] = 0u;
       }
-      if (!live) {
-        // nothing to store for a lane past the call's heads
-      } else if (n_split == 1) {
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(o_part) + orow + cc * 32;
+      if (n_split == 1) {
 #pragma unroll
-        for (int t = 0; t < 32; t += 8) {
-          const uint4 v = make_uint4(pack_bf16x2(__uint_as_float(ov[t]) * inv, __uint_as_float(ov[t + 1]) * inv),
-                                     pack_bf16x2(__uint_as_float(ov[t + 2]) * inv, __uint_as_float(ov[t + 3]) * inv),
-                                     pack_bf16x2(__uint_as_float(ov[t + 4]) * inv, __uint_as_float(ov[t + 5]) * inv),
-                                     pack_bf16x2(__uint_as_float(ov[t + 6]) * inv, __uint_as_float(ov[t + 7]) * inv));
-          *reinterpret_cast<uint4*>(dst + t) = v;
-        }
+        for (int t = 0; t < 32; t += 8)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + (uint32_t)(cc * 64 + t * 2)),
+                       "r"(pack_bf16x2(__uint_as_float(ov[t]) * inv, __uint_as_float(ov[t + 1]) * inv)),
+                       "r"(pack_bf16x2(__uint_as_float(ov[t + 2]) * inv, __uint_as_float(ov[t + 3]) * inv)),
+                       "r"(pack_bf16x2(__uint_as_float(ov[t + 4]) * inv, __uint_as_float(ov[t + 5]) * inv)),
+                       "r"(pack_bf16x2(__uint_as_float(ov[t + 6]) * inv, __uint_as_float(ov[t + 7]) * inv))
+                       : "memory");
       } else {
-        float* dst = reinterpret_cast<float*>(o_part) + orow + cc * 32;
 #pragma unroll
-        for (int t = 0; t < 32; t += 4) {
-          const float4 v = make_float4(__uint_as_float(ov[t]) * inv, __uint_as_float(ov[t + 1]) * inv,
-                                       __uint_as_float(ov[t + 2]) * inv, __uint_as_float(ov[t + 3]) * inv);
-          *reinterpret_cast<float4*>(dst + t) = v;
-        }
+        for (int t = 0; t < 32; t += 4)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + (uint32_t)(cc * 128 + t * 4)),
+                       "r"(__float_as_uint(__uint_as_float(ov[t]) * inv)),
+                       "r"(__float_as_uint(__uint_as_float(ov[t + 1]) * inv)),
+                       "r"(__float_as_uint(__uint_as_float(ov[t + 2]) * inv)),
+                       "r"(__float_as_uint(__uint_as_float(ov[t + 3]) * inv))
+                       : "memory");
       }
+    }
+    if (live) {
+      fence_proxy_async_smem();  // the staged row, visible to the bulk copy
+      uint8_t* dst = static_cast<uint8_t*>(o_part) + orow * (n_split == 1 ? 2 : 4);
+      bulk_store(dst, stg, row_bytes);
+      bulk_commit();
+      bulk_wait_all();
     }
     if (rank == 0 && grp == 0 && live) {
       lse_part[((size_t)b * n_split + split) * n_heads + i] =
@@ -837,7 +902,11 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
   __syncthreads();
   tc_fence_after();
 #ifdef MLA_TRACE
-  if (rank == 0 && tid == 0 && unit < 4096) g_mla_cluster_ns[2 * unit + 1] = global_timer_ns();
+  if (tid == 0) {
+    MLA_CLUSTER_STAMP(kCeEnd);
+    if (rank == 0 && unit < kTraceClusters)
+      g_mla_cluster_ns[unit * kClusterEvents + kCeClocks] = (unsigned long long)(clock64() - clk_start);
+  }
 #endif
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
   cluster_sync();
@@ -889,6 +958,7 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
   const uint32_t tmem_cols = n_tile <= 32 ? 32u : 64u;
 
   if (tid == 0) {
+    MLA_KERNEL_STAMP_MIN(kKeCombineStart);
     *abort_flag = 0;
     for (int kb = 0; kb < 8; ++kb) mbar_init(bar_k(kb), 1);
     mbar_init(bar_mma, 1);
@@ -913,6 +983,10 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
   }
   grid_dep_launch();  // a programmatically dependent successor (the output projection) may start
   grid_dep_wait();    // o_part / lse_part come from the attention kernel
+  if (tid == 0) {
+    MLA_KERNEL_STAMP_MAX(kKeCombineWaited);
+    MLA_KERNEL_STAMP_MIN(kKeCombineFirstWaited);
+  }
 
   if (n_split == 1) {
     // O~ rows b0.. of head h: eight boxes of 64 columns x n_tile rows (rows
@@ -981,12 +1055,14 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
       }
     }
     mma_commit(bar_mma);
+    MLA_KERNEL_STAMP_MAX(kKeCombineIssued);
   }
   __syncwarp();
 
   if (warp < 4) {
     wait(bar_mma, 0, ab);
     tc_fence_after();
+    if (tid == 0) MLA_KERNEL_STAMP_MAX(kKeCombineMmaDone);
     const int e = warp * 32 + lane;  // value dimension
     for (int n0 = 0; n0 < n_tile; n0 += 16) {
       uint32_t v[16];
@@ -1002,6 +1078,7 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, tmem_cols);
+  if (tid == 0) MLA_KERNEL_STAMP_MAX(kKeCombineEnd);
 }
 
 }  // namespace mla

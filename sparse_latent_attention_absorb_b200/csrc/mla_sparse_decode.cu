@@ -585,11 +585,29 @@ extern "C" int mla_trace_fetch(long long* host, int n) {
   return cudaMemcpyFromSymbol(host, g_mla_trace, sizeof(long long) * total) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// Trace builds only: start and end (globaltimer ns) of every cluster of the
-// last traced launch, 2 x 4096 values.
+// Trace builds only: clears the whole-kernel stamps (earliest-start slots to
+// the largest value, latest-end slots to zero).
+extern "C" int mla_trace_reset() {
+  unsigned long long v[kKernelEvents];
+  for (int e = 0; e < kKernelEvents; ++e)
+    v[e] = (e == kKeAbsorbStart || e == kKeCombineStart || e == kKeCombineFirstWaited) ? ~0ull : 0ull;
+  return cudaMemcpyToSymbol(g_mla_kernel_ns, v, sizeof(v)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// Trace builds only: the whole-kernel stamps (kKernelEvents values).
+extern "C" int mla_trace_kernel_fetch(unsigned long long* host, int n) {
+  if (!host || n < kKernelEvents) return MLA_ERR_INVALID_ARG;
+  return cudaMemcpyFromSymbol(host, g_mla_kernel_ns, sizeof(unsigned long long) * kKernelEvents) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
+}
+
+// Trace builds only: the milestones of every cluster of the last traced
+// launch (kClusterEvents values per cluster, 4096 clusters).
 extern "C" int mla_trace_cluster_fetch(unsigned long long* host, int n) {
-  if (!host || n < 2 * 4096) return MLA_ERR_INVALID_ARG;
-  return cudaMemcpyFromSymbol(host, g_mla_cluster_ns, sizeof(unsigned long long) * 2 * 4096) == cudaSuccess
+  const int total = kClusterEvents * kTraceClusters;
+  if (!host || n < total) return MLA_ERR_INVALID_ARG;
+  return cudaMemcpyFromSymbol(host, g_mla_cluster_ns, sizeof(unsigned long long) * total) == cudaSuccess
              ? MLA_OK
              : MLA_ERR_CUDA;
 }
