@@ -334,6 +334,9 @@ enum ClusterEvent {
   kCePvDone,       // softmax: last PV complete (epilogue may read O)
   kCeEnd,          // every thread past the epilogue
   kCeClocks,       // SM clock cycles from kCeStart to kCeEnd (clock64)
+  kCeDepWaited,    // softmax: past the wait on the absorption kernel
+  kCeQueryLoaded,  // softmax: first part of the query half in registers
+  kCeFirstIssued,  // gather warp 0: first tile's copies issued
   kClusterEvents
 };
 constexpr int kTraceClusters = 4096;
@@ -481,6 +484,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       }
       cp_async_commit();
       if (lane == 0) MLA_TRACE_STAMP(kTrGatherIssue, j);
+      if (j == 0 && g == 0 && lane == 0) MLA_CLUSTER_STAMP(kCeFirstIssued);
       const uint32_t valid = (__ballot_sync(0xffffffffu, idx >= 0) >> (16 * h)) & 0xffffu;
       cp_async_wait_all();
       fence_proxy_async_smem();
@@ -607,6 +611,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     // memory as a 64B-swizzled K-major row.
     {
       grid_dep_wait();  // q_lat comes from the absorption kernel
+      if (leader && grp == 0) MLA_CLUSTER_STAMP(kCeDepWaited);
       const uint4* ql = reinterpret_cast<const uint4*>(q_lat + ((size_t)b * n_heads + (live ? i : 0)) * kDl + rank * 256);
 #pragma unroll
       for (int part = 0; part < 2; ++part) {  // 64 latent values = 32 columns each
@@ -616,7 +621,8 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
           const uint4 x = live ? __ldg(ql + (2 * grp + part) * 8 + v) : make_uint4(0u, 0u, 0u, 0u);
           r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
         }
-        tmem_st32(tmem + lane_base + kColQ + (2 * grp + part) * 32, r);
+        tmem_st32(tmem + lane_base + kColQ + (2 * grp + part) * 32, r);  // waits for the loads
+        if (part == 0 && leader && grp == 0) MLA_CLUSTER_STAMP(kCeQueryLoaded);
       }
       tmem_wait_st();
       tc_fence_before();
