@@ -894,7 +894,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       uint8_t* dst = static_cast<uint8_t*>(o_part) + orow * (n_split == 1 ? 2 : 4);
       bulk_store(dst, stg, row_bytes);
       bulk_commit();
-      bulk_wait_all();
+      bulk_wait_read();
     }
     if (rank == 0 && grp == 0 && live) {
       lse_part[((size_t)b * n_split + split) * n_heads + i] =
