@@ -418,10 +418,9 @@ def gpu_arm(args, rank, world, device):
     # that read only half of wkv_b each, enough wkv_b copies that a rotation of
     # the halves they read exceeds L2
     q_lat = [torch.empty((B, 128, 512), dtype=torch.bfloat16, device=device) for _ in sets]
-    # the attention kernel's per-split output: f32 partials, or the bf16 mixed
-    # latent when each row is a single split
-    o_part = (torch.empty((B, 128, 512), dtype=torch.bfloat16, device=device) if n_split == 1 else
-              torch.empty((B, n_split, 128, 512), dtype=torch.float32, device=device))
+    # the attention kernel's per-split output (bf16; the mixed latent itself
+    # when each row is a single split)
+    o_part = torch.empty((B, n_split, 128, 512), dtype=torch.bfloat16, device=device)
     lse_part = torch.empty((B, n_split, 128), dtype=torch.float32, device=device)
     n_w = max(len(sets), math.ceil(2 * L2_BYTES / (128 * 128 * 512 * 2)))
     w_copies = [sets[i]["wkv_b"] if i < len(sets) else torch.empty_like(sets[0]["wkv_b"]).copy_(sets[i % len(sets)]["wkv_b"])

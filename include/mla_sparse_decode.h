@@ -89,9 +89,8 @@ int mla_num_splits(int B, int K);
 
 /* Bytes of scratch `mla_sparse_decode` needs for these sizes on the current
  * device: the absorbed queries (bf16 [B,128,512]), the per-split outputs of
- * mla_sparse_attend (see there: f32 [B,splits,128,512], or bf16 [B,128,512]
- * with one split) and their log-sum-exps (f32 [B,splits,128]).  Returns 0 for
- * invalid sizes. */
+ * mla_sparse_attend (see there: bf16 [B,splits,128,512]) and their
+ * log-sum-exps (f32 [B,splits,128]).  Returns 0 for invalid sizes. */
 size_t mla_sparse_decode_workspace_size(int B, int K, int S_max);
 
 /*
@@ -135,11 +134,11 @@ int mla_absorb_q(const void* q_nope, const void* wkv_b, void* q_lat, int B, cuda
  * Steps "scores" .. "mix" for every (row, split) (model.py 596-605), the
  * key positions of row b being split into `n_split` contiguous ranges of index
  * slots:
- *   o_part           n_split > 1: f32 [B,n_split,128,512], o_part[b,s,h,:] =
+ *   o_part           bf16 [B,n_split,128,512], o_part[b,s,h,:] = the
  *                    softmax-normalised mix of the cached latents over the
- *                    valid positions of split s;
- *                    n_split == 1: bf16 [B,128,512], the mixed latent
- *                    O~[b,h,:] itself (rounded to bf16, the value-up operand)
+ *                    valid positions of split s, rounded to bf16; with
+ *                    n_split == 1 ([B,128,512]) it is the mixed latent
+ *                    O~[b,h,:] itself, the value-up operand
  *   lse_part[b,s,h]  f32 [B,n_split,128]      log-sum-exp of the split's
  *                    scaled scores (-inf when the split has no valid index)
  *   q_lat bf16 [B,128,512] (from mla_absorb_q), the other inputs as above.
@@ -152,7 +151,7 @@ int mla_sparse_attend(const void* q_lat, const void* q_pe, const void* kv_cache,
 /*
  * Steps "combine" and "value-up" (model.py 605-606), o_part and lse_part in
  * the layout mla_sparse_attend writes for this n_split:
- *   O~[b,h,:] = sum_s exp(lse_part[b,s,h] - L) o_part[b,s,h,:],
+ *   O~[b,h,:] = sum_s exp(lse_part[b,s,h] - L) o_part[b,s,h,:]   (in f32),
  *   L = log sum_s exp(lse_part[b,s,h])          (n_split > 1; with one split
  *                                                O~ = o_part, L = lse_part),
  *   out[b,h,e] = bf16( sum_c bf16(O~[b,h,c]) * wkv_b[h*256 + 128 + e, c] ),

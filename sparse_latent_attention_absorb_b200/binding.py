@@ -208,14 +208,14 @@ def _o_part_spec(B: int, n_split: int):
     """Shape and dtype of mla_sparse_attend's o_part for this split count."""
     if n_split == 1:
         return (B, H, D_LAT), torch.bfloat16
-    return (B, n_split, H, D_LAT), torch.float32
+    return (B, n_split, H, D_LAT), torch.bfloat16
 
 
 def mla_sparse_attend(q_lat, q_pe, kv_cache, pe_cache, end_pos, topk_idx, scale, o_part=None, lse_part=None,
                       d_status=None, stream=None):
     """Per-split outputs; returns (o_part, lse_part [B,S,128] f32).
 
-    o_part is f32 [B,S,128,512] (normalised mix per split) when S > 1, and the
+    o_part is bf16 [B,S,128,512] (normalised mix per split) when S > 1, and the
     bf16 mixed latent [B,128,512] when each row is one split (S == 1)."""
     lib = load_library()
     B, S_max, K = q_lat.shape[0], kv_cache.shape[1], topk_idx.shape[1]

@@ -851,13 +851,14 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       if (leader && grp == 0) MLA_CLUSTER_STAMP(kCePvDone);
     }
     const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-    // A row of one split is final here: its mixed latent O~ goes out in bf16
-    // (the value-up operand); several splits keep f32 partials for the merge.
+    // The split's normalised mix goes out in bf16: with one split per row it
+    // is the mixed latent O~ itself (the value-up operand); with several the
+    // value-up kernel merges the splits by their log-sum-exp weights.
     // The ring is idle once the last PV is done, so each thread stages its
     // 128-column half row there (rows padded by 16 bytes: the 32 rows of a
     // warp fall on distinct banks) and writes it out with one bulk copy.
     const size_t orow = (((size_t)b * n_split + split) * n_heads + (live ? i : 0)) * kDl + rank * 256 + 128 * grp;
-    const uint32_t row_bytes = n_split == 1 ? 128u * 2u : 128u * 4u;
+    constexpr uint32_t row_bytes = 128u * 2u;
     const uint32_t stg = sStage + (uint32_t)(grp * kH + i) * (row_bytes + 16u);
 #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {
@@ -869,29 +870,18 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
 #pragma unroll
         for (int t = 0; t < 32; ++t) ov[t] = 0u;
       }
-      if (n_split == 1) {
 #pragma unroll
-        for (int t = 0; t < 32; t += 8)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + (uint32_t)(cc * 64 + t * 2)),
-                       "r"(pack_bf16x2(__uint_as_float(ov[t]) * inv, __uint_as_float(ov[t + 1]) * inv)),
-                       "r"(pack_bf16x2(__uint_as_float(ov[t + 2]) * inv, __uint_as_float(ov[t + 3]) * inv)),
-                       "r"(pack_bf16x2(__uint_as_float(ov[t + 4]) * inv, __uint_as_float(ov[t + 5]) * inv)),
-                       "r"(pack_bf16x2(__uint_as_float(ov[t + 6]) * inv, __uint_as_float(ov[t + 7]) * inv))
-                       : "memory");
-      } else {
-#pragma unroll
-        for (int t = 0; t < 32; t += 4)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + (uint32_t)(cc * 128 + t * 4)),
-                       "r"(__float_as_uint(__uint_as_float(ov[t]) * inv)),
-                       "r"(__float_as_uint(__uint_as_float(ov[t + 1]) * inv)),
-                       "r"(__float_as_uint(__uint_as_float(ov[t + 2]) * inv)),
-                       "r"(__float_as_uint(__uint_as_float(ov[t + 3]) * inv))
-                       : "memory");
-      }
+      for (int t = 0; t < 32; t += 8)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + (uint32_t)(cc * 64 + t * 2)),
+                     "r"(pack_bf16x2(__uint_as_float(ov[t]) * inv, __uint_as_float(ov[t + 1]) * inv)),
+                     "r"(pack_bf16x2(__uint_as_float(ov[t + 2]) * inv, __uint_as_float(ov[t + 3]) * inv)),
+                     "r"(pack_bf16x2(__uint_as_float(ov[t + 4]) * inv, __uint_as_float(ov[t + 5]) * inv)),
+                     "r"(pack_bf16x2(__uint_as_float(ov[t + 6]) * inv, __uint_as_float(ov[t + 7]) * inv))
+                     : "memory");
     }
     if (live) {
       fence_proxy_async_smem();  // the staged row, visible to the bulk copy
-      uint8_t* dst = static_cast<uint8_t*>(o_part) + orow * (n_split == 1 ? 2 : 4);
+      uint8_t* dst = static_cast<uint8_t*>(o_part) + orow * 2;
       bulk_store(dst, stg, row_bytes);
       bulk_commit();
       bulk_wait_read();
@@ -922,7 +912,8 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
 //
 // Per (head h, tile of up to 64 rows b):
 //   with several splits: coefficients a_s = exp(lse_s - L) with
-//   L = log sum_s exp(lse_s); O~[b, :] = sum_s a_s o_part[b, s, h, :], rounded
+//   L = log sum_s exp(lse_s); O~[b, :] = sum_s a_s o_part[b, s, h, :] (bf16
+//   partials, summed in f32), rounded
 //   to bf16 into shared memory (K-major B operand, 128B-swizzled);
 //   with one split: O~ is already bf16 in memory and comes in by TMA;
 //   D[e, b] = sum_c W_UV[h, e, c] * O~[b, c]   (M = 128 value dims, K = 512)
@@ -1004,7 +995,6 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
     if (tid < rows && lse_out)
       lse_out[(size_t)(b0 + tid) * n_heads + h] = lse_part[(size_t)(b0 + tid) * n_heads + h];
   } else {
-    const float* o_f32 = static_cast<const float*>(o_part);
     // split weights, one row per thread
     if (tid < rows) {
       const int b = b0 + tid;
@@ -1023,20 +1013,34 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
     }
     __syncthreads();
 
-    // merged O~ rows -> bf16 K-major operand (row n = batch row, 512 columns)
+    // merged O~ rows -> bf16 K-major operand (row n = batch row, 512
+    // columns): each split's 8 columns are one 16-byte load, up to sixteen
+    // splits in flight together
+    const __nv_bfloat16* o_bf = static_cast<const __nv_bfloat16*>(o_part);
+    const size_t split_stride = (size_t)n_heads * kDl;
     for (int it = tid; it < n_tile * 64; it += kCombineThreads) {
       const int n = it >> 6, q = it & 63;  // q: 8-column chunk of the 512
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (n < rows) {
-        const int b = b0 + n;
-#pragma unroll 4
-        for (int s = 0; s < n_split; ++s) {
-          const float a = coef[n * kCombineMaxSplits + s];
-          const float4* src =
-              reinterpret_cast<const float4*>(o_f32 + (((size_t)b * n_split + s) * n_heads + h) * kDl + q * 8);
-          const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
-          acc[0] += a * x0.x; acc[1] += a * x0.y; acc[2] += a * x0.z; acc[3] += a * x0.w;
-          acc[4] += a * x1.x; acc[5] += a * x1.y; acc[6] += a * x1.z; acc[7] += a * x1.w;
+        const float* cf = coef + n * kCombineMaxSplits;
+        const __nv_bfloat16* src = o_bf + ((size_t)(b0 + n) * n_split * n_heads + h) * kDl + q * 8;
+        for (int s0 = 0; s0 < n_split; s0 += 16) {
+          uint4 x[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            if (s0 + u < n_split) x[u] = __ldg(reinterpret_cast<const uint4*>(src + (size_t)(s0 + u) * split_stride));
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            if (s0 + u < n_split) {
+              const float a = cf[s0 + u];
+              const uint32_t w[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {  // bf16 -> f32 is exact: the high half of the word
+                acc[2 * e] += a * __uint_as_float(w[e] << 16);
+                acc[2 * e + 1] += a * __uint_as_float(w[e] & 0xffff0000u);
+              }
+            }
+          }
         }
       }
       const uint32_t dst = sB + (q >> 3) * (n_tile * 128) + sw128_offset(n, q & 7);

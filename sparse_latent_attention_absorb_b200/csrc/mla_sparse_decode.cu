@@ -244,8 +244,8 @@ WorkspaceLayout workspace_layout(int B, int n_split, int n_heads = kH) {
   size_t off = 0;
   w.q_lat = off;
   off = round_up(off + (size_t)B * n_heads * kDl * 2, 256);
-  w.o_part = off;  // f32 partials per split, or bf16 O~ when a row is one split
-  off = round_up(off + (size_t)B * n_split * n_heads * kDl * (n_split == 1 ? 2 : 4), 256);
+  w.o_part = off;  // bf16: each split's normalised mix (O~ itself when a row is one split)
+  off = round_up(off + (size_t)B * n_split * n_heads * kDl * 2, 256);
   w.lse_part = off;
   off = round_up(off + (size_t)B * n_split * n_heads * 4, 256);
   w.total = off;

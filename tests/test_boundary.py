@@ -61,9 +61,9 @@ def test_workspace_size_formula(lib):
     for B, K in ((1, 256), (8, 2048), (64, 2048), (3, 100)):
         n = lib.mla_num_splits(B, K)
         got = lib.mla_sparse_decode_workspace_size(B, K, 4096)
-        # q_lat bf16, per-split outputs (f32 partials, or bf16 O~ with one
-        # split), their log-sum-exps
-        o_bytes = B * 128 * 512 * 2 if n == 1 else B * n * 128 * 512 * 4
+        # q_lat bf16, per-split outputs (bf16; O~ itself with one split),
+        # their log-sum-exps
+        o_bytes = B * n * 128 * 512 * 2
         need = B * 128 * 512 * 2 + o_bytes + B * n * 128 * 4
         assert need <= got <= need + 3 * 256
     assert lib.mla_sparse_decode_workspace_size(0, 1, 1) == 0

@@ -151,11 +151,11 @@ def test_combine_step_single_split(B):
 
 
 def test_combine_step_with_given_partials():
-    """Steps a6-a7 alone on synthetic partials: exact LSE weights, then the
-    W_UV product of the bf16-rounded mix."""
+    """Steps a6-a7 alone on synthetic bf16 partials: exact LSE weights, then
+    the W_UV product of the bf16-rounded mix."""
     gen = torch.Generator().manual_seed(5)
     B, S = 7, 3  # the combine entry point accepts any split count in [1, 128]
-    o_part = torch.randn((B, S, 128, 512), generator=gen, dtype=torch.float32) * 0.05
+    o_part = (torch.randn((B, S, 128, 512), generator=gen, dtype=torch.float32) * 0.05).to(torch.bfloat16)
     lse_part = torch.randn((B, S, 128), generator=gen, dtype=torch.float32) * 3
     lse_part[0, :, 5] = float("-inf")          # a row-head with no valid position
     wkv_b = (torch.randn((128 * 256, 512), generator=gen) * 512 ** -0.5).to(torch.bfloat16)
