@@ -401,6 +401,30 @@ int mla_output_projection_shard(const void* x, const void* wo, long long ld_wo, 
                                 void* workspace, size_t workspace_bytes, int* d_status, cudaStream_t stream);
 
 /*
+ * The output projection from a prepared copy of wo (the same projection as
+ * mla_output_projection_shard, bit for bit).  Read in place, each work unit
+ * of the projection touches 512 bytes in each of 128 rows of wo 32 KB apart;
+ * the prepared copy holds every such unit's 64 KB contiguously, so the
+ * weight stream runs closer to the HBM copy rate.  Prepare once per weight
+ * (like the fp8 dequantisation of wkv_b), project every step:
+ *   mla_prepare_wo(wo, ld_wo, dim, k_in, wo_prepared, stream)
+ *     wo           bf16 rows of ld_wo elements (16-byte aligned, ld_wo a
+ *                  multiple of 8 and >= k_in); columns [0, k_in) are used
+ *     wo_prepared  device buffer of dim * k_in * 2 bytes, 16-byte aligned,
+ *                  written in an internal layout (only the function below
+ *                  reads it); enqueued on `stream`
+ *     dim  a multiple of 128, 128 <= dim <= 65536
+ *     k_in a multiple of 256, 256 <= k_in <= 16384
+ *   mla_output_projection_prepared(x, wo_prepared, delta, B, dim, k_in, ...)
+ *     x bf16 [B, k_in], delta bf16 [B, dim], workspace as
+ *     mla_output_projection_shard_workspace_size(B, dim, k_in).
+ * Both return an mla_status.
+ */
+int mla_prepare_wo(const void* wo, long long ld_wo, int dim, int k_in, void* wo_prepared, cudaStream_t stream);
+int mla_output_projection_prepared(const void* x, const void* wo_prepared, void* delta, int B, int dim, int k_in,
+                                   void* workspace, size_t workspace_bytes, int* d_status, cudaStream_t stream);
+
+/*
  * Self-test of the bounded waits every kernel relies on (no counterpart on the
  * pages): launches one CTA whose thread waits, through the kernels' own wait,
  * on a barrier that nothing arrives on.  After the wait limit (2 s) it must

@@ -29,7 +29,8 @@ EXPORTS = ("mla_status_string", "mla_num_splits", "mla_sparse_decode_workspace_s
            "mla_sparse_decode_project_workspace_size", "mla_sparse_decode_project", "mla_sparse_prefill",
            "mla_selftest_wait_timeout", "mla_check_topk_indices", "mla_set_index_checks",
            "mla_sparse_decode_heads_workspace_size", "mla_sparse_decode_heads",
-           "mla_output_projection_shard_workspace_size", "mla_output_projection_shard", "mla_dequant_fp8_blocks")
+           "mla_output_projection_shard_workspace_size", "mla_output_projection_shard", "mla_dequant_fp8_blocks",
+           "mla_prepare_wo", "mla_output_projection_prepared")
 STATIC_SCRATCH_BYTES = 32 << 20  # MLA_STATIC_SCRATCH_BYTES
 
 _lib = None
@@ -96,6 +97,10 @@ def load_library():
     lib.mla_dequant_fp8_blocks.argtypes = [p, p, p, i, i, p]
     lib.mla_output_projection_shard.restype = i
     lib.mla_output_projection_shard.argtypes = [p, p, ctypes.c_longlong, p, i, i, i, p, sz, p, p]
+    lib.mla_prepare_wo.restype = i
+    lib.mla_prepare_wo.argtypes = [p, ctypes.c_longlong, i, i, p, p]
+    lib.mla_output_projection_prepared.restype = i
+    lib.mla_output_projection_prepared.argtypes = [p, p, p, i, i, i, p, sz, p, p]
     lib.mla_selftest_wait_timeout.restype = i
     lib.mla_selftest_wait_timeout.argtypes = [p, p, p]
     _lib = lib
@@ -519,6 +524,49 @@ def mla_output_projection_shard(x, wo, delta=None, workspace=None, d_status=None
     rc = lib.mla_output_projection_shard(_ptr(x), _ptr(wo), wo.stride(0), _ptr(delta), B, dim, k_in, _ptr(workspace),
                                          workspace.numel(), _ptr(d_status), _stream(stream))
     _raise(rc, "mla_output_projection_shard")
+    return delta
+
+
+class PreparedWo:
+    """wo [dim, k_in] in the layout mla_output_projection_prepared streams
+    (built once per weight by mla_prepare_wo): `data` is a bf16 device buffer
+    of dim * k_in elements whose order is internal to the library."""
+
+    def __init__(self, data, dim: int, k_in: int):
+        self.data, self.dim, self.k_in = data, dim, k_in
+
+
+def mla_prepare_wo(wo, stream=None) -> PreparedWo:
+    """The prepared copy of wo, a bf16 [dim, k_in] CUDA view with unit column
+    stride (its rows may be strided: a tensor-parallel column slice)."""
+    lib = load_library()
+    if not (wo.is_cuda and wo.dtype == torch.bfloat16 and wo.dim() == 2 and wo.stride(1) == 1):
+        raise ValueError("wo: expected a CUDA bf16 [dim, k_in] view with unit column stride")
+    dim, k_in = wo.shape
+    data = torch.empty(dim * k_in, dtype=torch.bfloat16, device=wo.device)
+    _raise(lib.mla_prepare_wo(_ptr(wo), wo.stride(0), dim, k_in, _ptr(data), _stream(stream)), "mla_prepare_wo")
+    return PreparedWo(data, dim, k_in)
+
+
+def mla_output_projection_prepared(x, wo_p: PreparedWo, delta=None, workspace=None, d_status=None, stream=None):
+    """delta bf16 [B, dim] = x . wo^T from the prepared wo (bit-identical to
+    mla_output_projection_shard on the original); x bf16 [B, k_in]."""
+    lib = load_library()
+    B, k_in = x.shape
+    dim = wo_p.dim
+    _check(x, "x", torch.bfloat16, (B, wo_p.k_in))
+    if delta is None:
+        delta = torch.empty((B, dim), dtype=torch.bfloat16, device=x.device)
+    _check(delta, "delta", torch.bfloat16, (B, dim))
+    if workspace is None:
+        n = lib.mla_output_projection_shard_workspace_size(B, dim, k_in)
+        if n == 0:
+            raise MLAError(1, "mla_output_projection_shard_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=x.device)
+    _check(workspace, "workspace", torch.uint8)
+    rc = lib.mla_output_projection_prepared(_ptr(x), _ptr(wo_p.data), _ptr(delta), B, dim, k_in, _ptr(workspace),
+                                            workspace.numel(), _ptr(d_status), _stream(stream))
+    _raise(rc, "mla_output_projection_prepared")
     return delta
 
 

@@ -323,21 +323,29 @@ int launch_combine(const void* o_part, const float* lse_part, const void* wkv_b,
 // reduce kernel with a programmatic dependency on it.  With pdl, the
 // projection kernel itself depends programmatically on the kernel before it:
 // it requests its first weight stages before waiting for that kernel.
+// With `prepared`, wo is in the prepared layout (mla_prepare_wo) and is read
+// by bulk copies; its tensor maps are not used.
 int launch_projection(const void* x, const void* wo, void* delta, int B, int dim, const ProjPlan& p, void* partial,
-                      int* d_status, cudaStream_t stream, bool pdl, long long ld_wo = kProjK) {
+                      int* d_status, cudaStream_t stream, bool pdl, long long ld_wo = kProjK, bool prepared = false) {
   const int k_in = p.k_blocks * kProjKBlock;
   CUtensorMap tm_wo, tm_wo4, tm_x;
   int rc;
-  if ((rc = encode_wo(&tm_wo, wo, dim, k_in, ld_wo)) != MLA_OK) return rc;
-  if (p.kgroup == 1)
-    tm_wo4 = tm_wo;  // unused
-  else if ((rc = encode_wo4(&tm_wo4, wo, dim, k_in, ld_wo)) != MLA_OK)
-    return rc;
+  if (prepared) {
+    std::memset(&tm_wo, 0, sizeof(tm_wo));  // unused
+    tm_wo4 = tm_wo;
+  } else {
+    if ((rc = encode_wo(&tm_wo, wo, dim, k_in, ld_wo)) != MLA_OK) return rc;
+    if (p.kgroup == 1)
+      tm_wo4 = tm_wo;  // unused
+    else if ((rc = encode_wo4(&tm_wo4, wo, dim, k_in, ld_wo)) != MLA_OK)
+      return rc;
+  }
   if ((rc = encode_proj_x(&tm_x, x, B, p.n_tile, k_in)) != MLA_OK) return rc;
   if ((rc = launch_ex(projection_kernel, dim3((unsigned)p.n_ctas), dim3(kProjThreads),
                       proj_smem_bytes(p.n_tile, p.kgroup), stream, pdl, tm_wo, tm_wo4, tm_x,
-                      static_cast<float*>(partial), static_cast<__nv_bfloat16*>(delta), B, dim, p.n_tile, p.n_ctas,
-                      p.direct ? 1 : 0, p.kgroup, p.k_blocks, d_status)) != MLA_OK)
+                      static_cast<const __nv_bfloat16*>(prepared ? wo : nullptr), static_cast<float*>(partial),
+                      static_cast<__nv_bfloat16*>(delta), B, dim, p.n_tile, p.n_ctas, p.direct ? 1 : 0, p.kgroup,
+                      p.k_blocks, d_status)) != MLA_OK)
     return rc;
   if (p.direct) return MLA_OK;
   dim3 grid((unsigned)p.tiles, ceil_div(p.n_tile, kProjReduceRows));
@@ -790,6 +798,42 @@ extern "C" int mla_output_projection_shard(const void* x, const void* wo, long l
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
     return MLA_ERR_WORKSPACE;
   return launch_projection(x, wo, delta, B, dim, p, workspace, d_status, stream, false, ld_wo);
+}
+
+// wo in the prepared layout (see projection.cuh): one pass over it, once per
+// weight.
+extern "C" int mla_prepare_wo(const void* wo, long long ld_wo, int dim, int k_in, void* wo_prepared,
+                              cudaStream_t stream) {
+  if (!wo || !wo_prepared || !aligned16(wo) || !aligned16(wo_prepared)) return MLA_ERR_INVALID_ARG;
+  if (dim < kProjM || dim > kProjMaxDim || dim % kProjM) return MLA_ERR_INVALID_ARG;
+  if (k_in < kProjTileK || k_in > kProjK || k_in % kProjTileK) return MLA_ERR_INVALID_ARG;
+  if (ld_wo < k_in || ld_wo % 8 || ld_wo > (1LL << 31)) return MLA_ERR_INVALID_ARG;  // rows 16-byte aligned
+  DeviceInfo* info = nullptr;
+  int rc = current_device(&info);
+  if (rc != MLA_OK) return rc;
+  const long long chunks = (long long)dim * (k_in / 8);
+  const long long want = (chunks + 255) / 256;
+  const unsigned grid = (unsigned)(want < 8LL * info->sm_count ? want : 8LL * info->sm_count);
+  return launch_ex(prepare_wo_kernel, dim3(grid), dim3(256), 0, stream, false, static_cast<const uint4*>(wo),
+                   ld_wo / 8, dim, k_in, static_cast<uint4*>(wo_prepared));
+}
+
+extern "C" int mla_output_projection_prepared(const void* x, const void* wo_prepared, void* delta, int B, int dim,
+                                              int k_in, void* workspace, size_t workspace_bytes, int* d_status,
+                                              cudaStream_t stream) {
+  const void* ptrs[] = {x, wo_prepared, delta};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (!proj_sizes_ok(B, dim) || k_in < kProjTileK || k_in > kProjK || k_in % kProjTileK) return MLA_ERR_INVALID_ARG;
+  DeviceInfo* info = nullptr;
+  int rc = prepare(&info);
+  if (rc != MLA_OK) return rc;
+  const ProjPlan p = plan_projection(B, dim, info->sm_count, k_in);
+  const size_t need = p.partial_bytes > 0 ? p.partial_bytes : 256;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+    return MLA_ERR_WORKSPACE;
+  return launch_projection(x, wo_prepared, delta, B, dim, p, workspace, d_status, stream, false, kProjK, true);
 }
 
 // The decode step followed by the output projection: the workspace holds the

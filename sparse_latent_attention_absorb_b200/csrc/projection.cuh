@@ -32,6 +32,12 @@
 // Warp roles of projection_kernel (192 threads): warps 0-3 drain the
 // accumulator (TMEM lane quarter = warp), warp 4 lane 0 issues TMA, warp 5
 // allocates TMEM and its lane 0 issues the MMAs.
+//
+// A prepared wo (prepare_wo_kernel, once per weight) holds every 128 x 256
+// block of wo as 64 contiguous KB laid out exactly as the kernel's shared
+// memory wants it, so a work unit's weights arrive by one bulk copy: read in
+// place, the same unit touches 512 bytes in each of 128 rows 32 KB apart, and
+// the short runs cost DRAM bandwidth (each run opens a DRAM row for 512 bytes).
 #pragma once
 
 #include "kernels.cuh"
@@ -48,6 +54,7 @@ constexpr int kProjStagesMax = 8;
 constexpr int kProjStageBudget = 200 * 1024;       // shared memory for the ring
 constexpr int kProjABytes = kProjM * kProjKBlock * 2;  // 16 KB
 constexpr int kProjThreads = 192;
+constexpr int kProjTileK = 4 * kProjKBlock;        // columns of one prepared block (64 KB)
 constexpr int kProjReduceRows = 16;                // batch rows per reduce CTA
 
 // A unit covers kgroup consecutive k-blocks: 1, or kProjKGroupWide when the
@@ -79,11 +86,33 @@ constexpr int proj_smem_max() {
 static_assert(proj_smem_max() <= 232448, "shared memory");
 static_assert(proj_stages(kProjNMax, 1) >= 2 && proj_stages(kProjWideNMax, kProjKGroupWide) >= 2, "ring depth");
 
+// The prepared layout of wo [dim, k_in] (dim % 128 == 0, k_in % 256 == 0):
+// block (m, g) = rows [128 m, 128 m + 128) x columns [256 g, 256 g + 256),
+// at ((m * (k_in / 256)) + g) * 64 KB; inside it, 64-column k-block j at
+// j * 16 KB, 8-row group r at r * 1 KB, row i of the group at i * 128 B and
+// its 16-byte chunk q (columns 8q .. 8q + 7 of the k-block) at (q ^ i) * 16 B
+// (the 128-byte swizzle of a K-major UMMA operand).  One thread per chunk.
+__global__ void __launch_bounds__(256)
+prepare_wo_kernel(const uint4* __restrict__ wo, long long ld_chunks, int dim, int k_in, uint4* __restrict__ out) {
+  const long long row_chunks = k_in / 8;
+  const long long n = (long long)dim * row_chunks;
+  const long long blocks_per_row = k_in / kProjTileK;
+  for (long long c = blockIdx.x * (long long)blockDim.x + threadIdx.x; c < n; c += (long long)gridDim.x * blockDim.x) {
+    const long long row = c / row_chunks;
+    const int qa = (int)(c - row * row_chunks);  // chunk within the row
+    const long long m = row / kProjM;
+    const int rr = (int)(row - m * kProjM), r = rr >> 3, i = rr & 7;
+    const int g = qa >> 5, j = (qa >> 3) & 3, q = qa & 7;
+    const long long dst = (m * blocks_per_row + g) * 4096 + j * 1024 + r * 64 + i * 8 + (q ^ i);
+    out[dst] = wo[row * ld_chunks + qa];
+  }
+}
+
 __global__ void __launch_bounds__(kProjThreads, 1)
 projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_wo4,
-                  const __grid_constant__ CUtensorMap tm_x, float* __restrict__ partial,
-                  __nv_bfloat16* __restrict__ delta, int B, int dim, int n_tile, int n_ctas, int direct, int kgroup,
-                  int k_blocks, int* d_status) {
+                  const __grid_constant__ CUtensorMap tm_x, const __nv_bfloat16* __restrict__ wo_prepared,
+                  float* __restrict__ partial, __nv_bfloat16* __restrict__ delta, int B, int dim, int n_tile,
+                  int n_ctas, int direct, int kgroup, int k_blocks, int* d_status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -107,7 +136,13 @@ projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_consta
   // [group][k-block][row][128 B]: 8-row x 128-byte swizzle atoms, the groups
   // 4 KB apart, k-block j at j KB
   auto load_wo = [&](uint32_t dst, uint32_t bar, long long u) {
-    if (kgroup == 1)
+    if (wo_prepared != nullptr) {  // kgroup k-blocks of one prepared block, contiguous
+      const int kb0 = unit_kb0(u);
+      const __nv_bfloat16* src = wo_prepared +
+                                 ((size_t)unit_m(u) * (k_blocks / 4) + kb0 / 4) * (size_t)(kProjM * kProjTileK) +
+                                 (size_t)(kb0 % 4) * (kProjM * kProjKBlock);
+      bulk_load(dst, src, (uint32_t)(kgroup * kProjABytes), bar);
+    } else if (kgroup == 1)
       tma_load_2d(dst, &tm_wo, bar, unit_kb0(u) * kProjKBlock, unit_m(u) * kProjM);
     else
       tma_load_4d(dst, &tm_wo4, bar, 0, 0, unit_kb0(u), unit_m(u) * (kProjM / 8));
@@ -153,7 +188,7 @@ projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_consta
   if (warp == 4) {
     // ------------------------------------------------------------ TMA
     if (lane == 0 && n_units > 0) {
-      tma_prefetch_desc(kgroup == 1 ? &tm_wo : &tm_wo4);
+      if (wo_prepared == nullptr) tma_prefetch_desc(kgroup == 1 ? &tm_wo : &tm_wo4);
       tma_prefetch_desc(&tm_x);
       // The first stages' weights go out before the wait on the kernel that
       // writes x (programmatic dependent launch): wo does not depend on it.
@@ -189,13 +224,15 @@ projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_consta
         tc_fence_after();
         const uint32_t a0 = sRing + st * stage_bytes;
         const uint32_t b0 = a0 + a_bytes;
-        // wo k-block j: the 2-D box (8-row groups 1 KB apart), or block j of
-        // the 4-D box (groups 4 KB apart, block j at j KB)
-        const uint32_t a_sbo = kgroup == 1 ? 1024u : 4096u;
+        // wo k-block j: the 2-D box (8-row groups 1 KB apart), block j of
+        // the 4-D box (groups kgroup KB apart, block j at j KB), or k-block j
+        // of a prepared block (groups 1 KB apart, block j at j * 16 KB)
+        const uint32_t a_sbo = wo_prepared != nullptr ? 1024u : 1024u * (uint32_t)kgroup;
+        const uint32_t a_jstride = wo_prepared != nullptr ? (uint32_t)kProjABytes : 1024u;
         for (int j = 0; j < kgroup; ++j) {
 #pragma unroll
           for (int k = 0; k < kProjKBlock / 16; ++k) {  // 32 bytes of k per step inside the 128-byte rows
-            const uint64_t a = smem_desc_sw128(a0 + j * 1024 + k * 32, 16, a_sbo);
+            const uint64_t a = smem_desc_sw128(a0 + j * a_jstride + k * 32, 16, a_sbo);
             const uint64_t bd = smem_desc_sw128(b0 + j * n_tile * kProjKBlock * 2 + k * 32, 16, 1024);
             mma_ss(tmem + acc * acc_cols, a, bd, idesc, (first && j == 0 && k == 0) ? 0u : 1u);
           }

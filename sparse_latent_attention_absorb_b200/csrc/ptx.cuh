@@ -183,6 +183,15 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // Named barrier over `count` threads (a multiple of 32) of this CTA.
+// Bulk copy of `bytes` (a multiple of 16) from global memory into this CTA's
+// shared memory (both addresses 16-byte aligned), completing on mbarrier
+// `bar` as transaction bytes.  No multicast.
+__device__ __forceinline__ void bulk_load(uint32_t sdst, const void* gsrc, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(sdst),
+               "l"(gsrc), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 // Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory to
 // global memory (both addresses 16-byte aligned), in the thread's bulk group.
 __device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {

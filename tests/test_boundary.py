@@ -278,3 +278,28 @@ def test_dequant_rejects_bad_arguments_without_a_launch(lib):
     assert call(rows=0) == INVALID_ARG
     assert call(cols=8) == INVALID_ARG
     assert call(cols=520 + 4) == INVALID_ARG
+
+
+def test_prepared_projection_rejects_bad_arguments_without_a_launch(lib):
+    A = 0x10000
+
+    def prep(wo=_fake(A), ld=16384, dim=7168, k_in=16384, out=_fake(A)):
+        return lib.mla_prepare_wo(wo, ld, dim, k_in, out, None)
+
+    assert prep(wo=None) == INVALID_ARG
+    assert prep(out=_fake(A + 8)) == INVALID_ARG
+    for dim in (0, 64, 100, (1 << 16) + 128):
+        assert prep(dim=dim) == INVALID_ARG
+    for k_in in (0, 64, 192, 16384 + 256):  # whole 256-column blocks only
+        assert prep(k_in=k_in) == INVALID_ARG
+    for ld in (16383, 16380, 1 << 32):
+        assert prep(ld=ld) == INVALID_ARG
+
+    def proj(B=4, dim=7168, k_in=16384, x=_fake(A), w=_fake(A)):
+        return lib.mla_output_projection_prepared(x, w, _fake(A), B, dim, k_in, _fake(A), 1 << 30, None, None)
+
+    for k_in in (0, 64, 320, 16384 + 256):
+        assert proj(k_in=k_in) == INVALID_ARG
+    assert proj(B=0) == INVALID_ARG
+    assert proj(dim=100) == INVALID_ARG
+    assert proj(w=_fake(A + 4)) == INVALID_ARG
