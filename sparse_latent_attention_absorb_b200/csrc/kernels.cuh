@@ -337,6 +337,9 @@ enum ClusterEvent {
   kCeDepWaited,    // softmax: past the wait on the absorption kernel
   kCeQueryLoaded,  // softmax: first part of the query half in registers
   kCeFirstIssued,  // gather warp 0: first tile's copies issued
+  kCeEntry,        // thread 0 at kernel entry
+  kCeEpLoaded,     // thread 0: end_pos of the row loaded
+  kCeIdxLoaded,    // gather warp 0: its first index word loaded
   kClusterEvents
 };
 constexpr int kTraceClusters = 4096;
@@ -379,8 +382,14 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
   const int k_begin = split * span;
   const int k_end = min(K, k_begin + span);
   const int n_tiles = k_end > k_begin ? (k_end - k_begin + kNt - 1) / kNt : 0;
+#ifdef MLA_TRACE
+  if (tid == 0) MLA_CLUSTER_STAMP(kCeEntry);
+#endif
   int ep = end_pos[b];
   ep = ep < 0 ? 0 : (ep > S_max ? S_max : ep);
+#ifdef MLA_TRACE
+  if (tid == 0 && ep >= 0) MLA_CLUSTER_STAMP(kCeEpLoaded);
+#endif
   // Cache slot of row b: b itself (decode), or cache_slot[b] when rows are
   // query positions sharing a sequence's latents (prefill).  A slot outside
   // [0, n_slots) leaves the row with no valid position (nothing is read).
@@ -510,6 +519,9 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     // loaded a pair ahead of its first use (a register copy of a pending load
     // would wait for the load)
     int cur = load_pair(0), nxt = load_pair(1), pf = load_pair(2);
+#ifdef MLA_TRACE
+    if (g == 0 && lane == 0 && cur != -2) MLA_CLUSTER_STAMP(kCeIdxLoaded);
+#endif
     for (int pr = 0; 2 * pr < n_tiles; ++pr) {
       gather_tile(2 * pr, cur, 0);
       prefetch_tile(pf, 0);
