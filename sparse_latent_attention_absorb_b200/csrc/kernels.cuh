@@ -64,6 +64,8 @@ enum KernelEvent {
   kKeCombineFirstWaited,  // min over CTAs: past the wait on the attention kernel
   kKeCombineIssued,    // max over CTAs: every k-block landed and its MMAs issued
   kKeCombineMmaDone,   // max over CTAs: accumulator complete
+  kKeCombineWeights,   // max over CTAs: split weights ready (several splits)
+  kKeCombineMerged,    // max over CTAs: merged operand in shared memory (several splits)
   kKernelEvents
 };
 #ifdef MLA_TRACE
@@ -534,14 +536,15 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
       pf = load_pair(pr + 3);
     }
     // With its last tile gathered (a few tiles before this CTA ends), gather
-    // warp 0 pulls W_UV of head blockIdx.x (+ gridDim.x ...) into L2 for the
-    // value-up kernel that follows (w_next = wkv_b, or null to skip).
-    if (g == 0 && lane == 0 && w_next != nullptr) {
-      for (int hh = blockIdx.x; hh < n_heads; hh += gridDim.x) {
-        const __nv_bfloat16* w = w_next + (size_t)(hh * kHeadRows + kDn) * kDl;  // 128 rows x 512: 128 KB
+    // warp 0 pulls W_UV of head blockIdx.x into L2 for the value-up kernel
+    // that follows (w_next = wkv_b, or null to skip).  One head at most: with
+    // fewer CTAs than heads the SMs left idle already run the value-up
+    // kernel's CTAs, which load W_UV themselves, and more prefetches per CTA
+    // only held up this CTA's exit (each bulk prefetch is issued in order).
+    if (g == 0 && lane == 0 && w_next != nullptr && (int)blockIdx.x < n_heads) {
+      const __nv_bfloat16* w = w_next + (size_t)(blockIdx.x * kHeadRows + kDn) * kDl;  // 128 rows x 512: 128 KB
 #pragma unroll
-        for (int part = 0; part < 4; ++part) prefetch_l2(w + part * 32 * kDl, 32 * kDl * 2);
-      }
+      for (int part = 0; part < 4; ++part) prefetch_l2(w + part * 32 * kDl, 32 * kDl * 2);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ QK issue
@@ -1024,6 +1027,7 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
       if (lse_out) lse_out[(size_t)b * n_heads + h] = total > 0.f ? mx + __logf(total) : -INFINITY;
     }
     __syncthreads();
+    if (tid == 0) MLA_KERNEL_STAMP_MAX(kKeCombineWeights);
 
     // merged O~ rows -> bf16 K-major operand (row n = batch row, 512
     // columns): each split's 8 columns are one 16-byte load, up to sixteen
@@ -1064,6 +1068,7 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
     fence_proxy_async_smem();
   }
   __syncthreads();
+  if (tid == 0 && n_split > 1) MLA_KERNEL_STAMP_MAX(kKeCombineMerged);
 
   if (tid == 0) {
     const uint32_t idesc = idesc_bf16_f32(128, n_tile, false, false);
