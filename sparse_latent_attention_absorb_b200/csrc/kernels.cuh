@@ -206,6 +206,7 @@ constexpr int kStages = 4;                         // gathered tile ring
 constexpr int kLatBlock = kNt * 128;               // one 64-column latent block of a tile (8 KB)
 constexpr int kStageBytes = 4 * kLatBlock + kNt * 64;  // 4 latent blocks + the rotary block: 36 KB
 constexpr int kQpeBytes = kH * 64;                 // rotary query columns of the half: 8 KB
+constexpr int kQBoxBytes = kH * 128;               // one 64-column box of the latent query half: 16 KB
 constexpr int kXHalves = (kNt / 8) * kH * 16;      // 16 KB: one exchanged score tile (fp16)
 constexpr int kXBytes = kXHalves + kH * 4;         // + each row's fp32 offset
 constexpr int kMslotBytes = 2 * kH * 4;            // running maximum published by each group
@@ -254,6 +255,7 @@ static_assert(kGatherWarps * 16 == kNt, "sixteen rows of a tile per gather warp"
 static_assert(kMmaWarp == kSoftmaxWarps && kPvWarp == kMmaWarp + 1 && kGatherWarp0 == kPvWarp + 1, "warp roles");
 
 struct AttendBars {
+  uint64_t q_tma;               // the query boxes (TMA, transaction bytes) landed
   uint64_t q_full;              // softmax warps (8 arrivals) after storing Q
   uint64_t kv_full[kStages];    // every gather warp (4 arrivals) once its copies of the tile landed
   uint64_t kv_empty[kStages];   // MMA commit after PV of the tile
@@ -367,7 +369,7 @@ __device__ unsigned long long g_mla_cluster_ns[kClusterEvents * kTraceClusters];
 #endif
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttendThreads, 1)
-sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat16* __restrict__ q_pe,
+sparse_attend_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant__ CUtensorMap tm_qpe,
                      const __nv_bfloat16* __restrict__ kv_cache, const __nv_bfloat16* __restrict__ pe_cache,
                      const int32_t* __restrict__ end_pos, const int32_t* __restrict__ topk_idx, float scale,
                      void* __restrict__ o_part, float* __restrict__ lse_part, int K, int S_max, int n_split,
@@ -417,6 +419,7 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
   if (tid == 0) {
     bars->abort_flag = 0;
     bars->qk_issued = 0;
+    mbar_init(smem_u32(&bars->q_tma), 1);
     mbar_init(smem_u32(&bars->q_full), kSoftmaxWarps);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&bars->kv_full[i]), kGatherWarps);
@@ -476,6 +479,8 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     auto gather_tile = [&](int j, int idx, int h) {
       const int st = j % kStages;
       if (j >= kStages) wait(smem_u32(&bars->kv_empty[st]), ((j / kStages) - 1) & 1, ab);
+      // stages 2 and 3 first hold the query's boxes, until it is in TMEM
+      if (j == 2) wait(smem_u32(&bars->q_full), 0, ab);
       if (lane == 0) MLA_TRACE_STAMP(kTrGatherWoke, j);
       const uint32_t stage = sStage + st * kStageBytes;
 #pragma unroll
@@ -548,6 +553,23 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ QK issue
+    // First the query: this CTA's latent half (four 64-column boxes of all
+    // 128 head rows, 128-byte swizzle) into ring stages 2 and 3, which the
+    // softmax warps copy into TMEM, and its 32 rotary columns straight into
+    // their K-major operand (64-byte swizzle).  Rows past the call's heads
+    // lie outside the tensor maps and arrive as zeros.
+    if (lane == 0 && n_tiles > 0) {
+      tma_prefetch_desc(&tm_qlat);
+      tma_prefetch_desc(&tm_qpe);
+      grid_dep_wait();  // q_lat comes from the absorption kernel
+      if (tid == kMmaWarp * 32) MLA_CLUSTER_STAMP(kCeDepWaited);
+      mbar_arrive_expect_tx(smem_u32(&bars->q_tma), 4 * kQBoxBytes + kQpeBytes);
+#pragma unroll
+      for (int bx = 0; bx < 4; ++bx)
+        tma_load_3d(sStage + (2 + bx / 2) * kStageBytes + (bx % 2) * kQBoxBytes, &tm_qlat,
+                    smem_u32(&bars->q_tma), (int)rank * 256 + bx * 64, 0, b);
+      tma_load_3d(sQpe, &tm_qpe, smem_u32(&bars->q_tma), (int)rank * 32, 0, b);
+    }
     // QK(j) as soon as its rows have landed and the previous tile's scores
     // have been read (one score buffer).
     if (lane == 0 && n_tiles > 0) {
@@ -622,35 +644,26 @@ sparse_attend_kernel(const __nv_bfloat16* __restrict__ q_lat, const __nv_bfloat1
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
 
     // This CTA's half of the query: latent columns 0..127 (group 0) and
-    // 128..255 (group 1) into TMEM; the 32 rotary values (group 1) into shared
-    // memory as a 64B-swizzled K-major row.
+    // 128..255 (group 1) from their staged boxes into TMEM (the rotary part
+    // is already in place); with no tile to process nothing is needed.
     {
-      grid_dep_wait();  // q_lat comes from the absorption kernel
-      if (leader && grp == 0) MLA_CLUSTER_STAMP(kCeDepWaited);
-      const uint4* ql = reinterpret_cast<const uint4*>(q_lat + ((size_t)b * n_heads + (live ? i : 0)) * kDl + rank * 256);
+      if (n_tiles > 0) {
+        wait(smem_u32(&bars->q_tma), 0, ab);
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {  // 64 latent values = 32 columns each
-        uint32_t r[32];
+        for (int part = 0; part < 2; ++part) {  // box 2 grp + part: 64 latent values = 32 columns
+          const uint32_t row = sStage + (2 + grp) * kStageBytes + part * kQBoxBytes + (uint32_t)i * 128u;
+          uint32_t r[32];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const uint4 x = live ? __ldg(ql + (2 * grp + part) * 8 + v) : make_uint4(0u, 0u, 0u, 0u);
-          r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
+          for (int v = 0; v < 8; ++v)
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(r[4 * v]), "=r"(r[4 * v + 1]), "=r"(r[4 * v + 2]), "=r"(r[4 * v + 3])
+                         : "r"(row + (uint32_t)((v ^ (i & 7)) << 4))
+                         : "memory");
+          tmem_st32(tmem + lane_base + kColQ + (2 * grp + part) * 32, r);
+          if (part == 0 && leader && grp == 0) MLA_CLUSTER_STAMP(kCeQueryLoaded);
         }
-        tmem_st32(tmem + lane_base + kColQ + (2 * grp + part) * 32, r);  // waits for the loads
-        if (part == 0 && leader && grp == 0) MLA_CLUSTER_STAMP(kCeQueryLoaded);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      if (grp == 1) {
-        const uint4* qp = reinterpret_cast<const uint4*>(q_pe + ((size_t)b * n_heads + (live ? i : 0)) * kDr + rank * 32);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint4 x = live ? __ldg(qp + v) : make_uint4(0u, 0u, 0u, 0u);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sQpe + sw64_offset(i, v)), "r"(x.x),
-                       "r"(x.y), "r"(x.z), "r"(x.w)
-                       : "memory");
-        }
-        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));

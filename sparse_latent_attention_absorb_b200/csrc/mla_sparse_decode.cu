@@ -121,6 +121,22 @@ int encode_q_nope(CUtensorMap* m, const void* q_nope, int B, int n_tile, int n_h
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// A per-head query tensor (q_lat: width 512, or q_pe: width 64) as a 3-D bf16
+// tensor {c: width, h: n_heads, b: B}, boxes of `box_c` columns x 128 heads x
+// 1 row: one box is a column block of all heads of a row (heads past n_heads
+// lie outside the tensor and read as zero).
+int encode_q_half(CUtensorMap* m, const void* q, int B, int n_heads, int width, int box_c,
+                  CUtensorMapSwizzle swizzle) {
+  cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)n_heads, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)width * 2, (cuuint64_t)n_heads * width * 2};
+  cuuint32_t box[3] = {(cuuint32_t)box_c, (cuuint32_t)kH, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
 // The mixed latent O~ (single-split rows) as a 3-D bf16 tensor
 // {c: 512, h: n_heads, b: B}, boxes of 64 c x 1 head x n_tile rows, 128-byte
 // swizzle (rows past B read as zero).
@@ -296,8 +312,12 @@ int launch_attend(const void* q_lat, const void* q_pe, const void* kv_cache, con
                   bool pdl, const int32_t* cache_slot = nullptr, int n_slots = 0, int n_heads = kH) {
   const long long ctas = 2LL * B * n_split;
   if (ctas > 0x7fffffffLL) return MLA_ERR_INVALID_ARG;
+  CUtensorMap tm_qlat, tm_qpe;
+  int rc;
+  if ((rc = encode_q_half(&tm_qlat, q_lat, B, n_heads, kDl, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK) return rc;
+  if ((rc = encode_q_half(&tm_qpe, q_pe, B, n_heads, kDr, 32, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK) return rc;
   return launch_ex(sparse_attend_kernel, dim3((unsigned)ctas), dim3(kAttendThreads), kAttendSmemBytes, stream, pdl,
-                   static_cast<const __nv_bfloat16*>(q_lat), static_cast<const __nv_bfloat16*>(q_pe),
+                   tm_qlat, tm_qpe,
                    static_cast<const __nv_bfloat16*>(kv_cache), static_cast<const __nv_bfloat16*>(pe_cache), end_pos,
                    topk_idx, scale, o_part, lse_part, K, S_max, n_split, span,
                    static_cast<const __nv_bfloat16*>(w_next), cache_slot, n_slots, n_heads, d_status);
