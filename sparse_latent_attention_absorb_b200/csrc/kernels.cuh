@@ -169,7 +169,9 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 // One 2-CTA cluster per (batch row b, key split s).  CTA rank r owns latent
 // columns [256r, 256r+256) and rotary columns [32r, 32r+32) of the score:
 //   * its half of the absorbed query is the A operand of QK: the 256 latent
-//     columns in TMEM (bf16 pairs), the 32 rotary columns in shared memory;
+//     columns in TMEM (bf16 pairs; four tensor-map boxes staged in ring
+//     stages 2-3, copied in by the softmax warps), the 32 rotary columns in
+//     shared memory (one tensor-map box, already the K-major operand);
 //   * for every selected position t of the split, a gather warp copies
 //     kv[b,t,its 256] (128B-swizzled rows) and pe[b,t,its 32] (64B-swizzled
 //     rows) into a ring of 64-position tiles (cp.async, 16 bytes per lane);
@@ -190,16 +192,17 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 //     group's TMEM buffer;
 //   * PV: O_r[h, its 256] += P[h,t] . kv[t, its 256]  (A = P from TMEM,
 //     B = the same gathered rows read M/N-major).
-// The split's normalised O and its log-sum-exp go to o_part / lse_part (O in
-// f32 per split; with a single split per row, the final O~ in bf16).
+// The split's normalised O (bf16; with a single split per row, the final O~)
+// and its log-sum-exp go to o_part / lse_part, O staged in the idle ring and
+// written by one bulk copy per thread.
 //
 // Warp roles (448 threads): warps 0-3 softmax group 0 (even tiles), warps
 // 4-7 softmax group 1 (odd tiles), warp w covering TMEM lanes 32(w%4)..;
-// warp 8 TMEM allocation + QK issue; warp 9 PV issue; warps 10-13 gather
-// (sixteen rows of every tile each).  QK and PV are issued by different
-// threads: their MMAs interleave in the tensor pipe, and a commit (which
-// tracks the issuing thread's MMAs only) signals PV completion without
-// waiting for a QK queued ahead of it.
+// warp 8 TMEM allocation, the query's tensor-map loads and QK issue; warp 9
+// PV issue; warps 10-13 gather (sixteen rows of every tile each).  QK and PV
+// are issued by different threads: their MMAs interleave in the tensor pipe,
+// and a commit (which tracks the issuing thread's MMAs only) signals PV
+// completion without waiting for a QK queued ahead of it.
 // =============================================================================
 constexpr int kNt = 64;                            // positions per tile
 constexpr int kStages = 4;                         // gathered tile ring
