@@ -86,6 +86,11 @@ SMALL_WORKLOADS = {
     "small_b80_ctx700_top300": Workload("small_b80_ctx700_top300", 80, 700, (700, 700), 300, "uniform", 2007),
     "small_b76_ctx150-2k_recent64_top700": Workload(
         "small_b76_ctx150-2k_recent64_top700", 76, 2048, (150, 2048), 700, "recent", 2008, recent=64),
+    # few rows, so each row's index slots are split over many clusters: 32
+    # and 18 key splits per row (the split merge reads them in batches of 16)
+    "small_b1_ctx4096_top2048": Workload("small_b1_ctx4096_top2048", 1, 4096, (4096, 4096), 2048, "uniform", 2009),
+    "small_b2_ctx1500-3k_top1100": Workload(
+        "small_b2_ctx1500-3k_top1100", 2, 3000, (1500, 3000), 1100, "uniform", 2010),
 }
 
 ALL_WORKLOADS = {**WORKLOADS, **SMALL_WORKLOADS}

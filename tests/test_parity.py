@@ -91,7 +91,8 @@ def test_decode_matches_oracle(name):
     assert int(status.item()) == 0
 
 
-@pytest.mark.parametrize("name", ["small_b4_ctx600-2k_recent128_top400", "small_b5_ctx40-700_top333"])
+@pytest.mark.parametrize("name", ["small_b4_ctx600-2k_recent128_top400", "small_b5_ctx40-700_top333",
+                                  "small_b1_ctx4096_top2048", "small_b2_ctx1500-3k_top1100"])
 def test_split_outputs_combine_to_oracle_mix(name):
     """Steps a2-a6: the per-split normalised mixes and log-sum-exps, merged in
     fp64 on the host, equal the oracle's mixed latent O~ and lse."""
@@ -150,11 +151,13 @@ def test_combine_step_single_split(B):
     assert np.array_equal(lse_out.cpu().numpy(), lse_part[:, 0].numpy())
 
 
-def test_combine_step_with_given_partials():
+@pytest.mark.parametrize("S", [3, 40])
+def test_combine_step_with_given_partials(S):
     """Steps a6-a7 alone on synthetic bf16 partials: exact LSE weights, then
-    the W_UV product of the bf16-rounded mix."""
-    gen = torch.Generator().manual_seed(5)
-    B, S = 7, 3  # the combine entry point accepts any split count in [1, 128]
+    the W_UV product of the bf16-rounded mix.  S = 40 takes the split loads
+    through three batches of sixteen, the last one ragged."""
+    gen = torch.Generator().manual_seed(5 + S)
+    B = 7  # the combine entry point accepts any split count in [1, 128]
     o_part = (torch.randn((B, S, 128, 512), generator=gen, dtype=torch.float32) * 0.05).to(torch.bfloat16)
     lse_part = torch.randn((B, S, 128), generator=gen, dtype=torch.float32) * 3
     lse_part[0, :, 5] = float("-inf")          # a row-head with no valid position
