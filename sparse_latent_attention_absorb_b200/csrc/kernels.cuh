@@ -129,14 +129,16 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
     wait(bar_load, 0, ab);
     tc_fence_after();
     const uint32_t idesc = idesc_bf16_f32(128, n_tile, /*a MN*/ true, /*b MN*/ false);
+    // descriptors built once; an operand at byte offset x is the base plus x/16
+    const uint64_t a0 = smem_desc_sw128(sA, 64 * 128 * 2, 1024);
+    const uint64_t b0d = smem_desc_sw128(sB, 16, 1024);
+#pragma unroll
     for (int k = 0; k < kDn / 16; ++k) {
       // A: 16 d-rows per step (two 8-row groups 1024 B apart); the two
-      // 64-wide c blocks are 16 KB apart.
-      const uint64_t a = smem_desc_sw128(sA + k * 16 * 128, 64 * 128 * 2, 1024);
-      // B: 32 bytes of d per step inside the 128-byte row; the second
-      // 64-wide d block follows the first.
-      const uint64_t b = smem_desc_sw128(sB + (k >> 2) * n_tile * 128 + (k & 3) * 32, 16, 1024);
-      mma_ss(tmem, a, b, idesc, k > 0 ? 1u : 0u);
+      // 64-wide c blocks are 16 KB apart.  B: 32 bytes of d per step inside
+      // the 128-byte row; the second 64-wide d block follows the first.
+      mma_ss(tmem, a0 + (uint64_t)((k * 16 * 128) >> 4),
+             b0d + (uint64_t)(((k >> 2) * n_tile * 128 + (k & 3) * 32) >> 4), idesc, k > 0 ? 1u : 0u);
     }
     mma_commit(bar_mma);
   }
@@ -1088,14 +1090,17 @@ combine_value_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_c
 
   if (tid == 0) {
     const uint32_t idesc = idesc_bf16_f32(128, n_tile, false, false);
+    // descriptors built once; an operand at byte offset x is the base plus x/16
+    const uint64_t a0 = smem_desc_sw128(sA, 16, 1024);
+    const uint64_t b0d = smem_desc_sw128(sB, 16, 1024);
     for (int kb = 0; kb < 8; ++kb) {  // each 64-column k-block as soon as it has landed
       wait(bar_k(kb), 0, ab);
       tc_fence_after();
-      for (int k = 4 * kb; k < 4 * kb + 4; ++k) {
-        const uint64_t a = smem_desc_sw128(sA + (k >> 2) * (128 * 128) + (k & 3) * 32, 16, 1024);
-        const uint64_t bd = smem_desc_sw128(sB + (k >> 2) * (n_tile * 128) + (k & 3) * 32, 16, 1024);
-        mma_ss(tmem, a, bd, idesc, k > 0 ? 1u : 0u);
-      }
+      const uint64_t ak = a0 + (uint64_t)((kb * (128 * 128)) >> 4);
+      const uint64_t bk = b0d + (uint64_t)((kb * (n_tile * 128)) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ss(tmem, ak + (uint64_t)(kk * 2), bk + (uint64_t)(kk * 2), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
     }
     mma_commit(bar_mma);
     MLA_KERNEL_STAMP_MAX(kKeCombineIssued);

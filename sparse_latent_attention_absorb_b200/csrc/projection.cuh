@@ -229,13 +229,17 @@ projection_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_consta
         // of a prepared block (groups 1 KB apart, block j at j * 16 KB)
         const uint32_t a_sbo = wo_prepared != nullptr ? 1024u : 1024u * (uint32_t)kgroup;
         const uint32_t a_jstride = wo_prepared != nullptr ? (uint32_t)kProjABytes : 1024u;
+        // descriptors built once per unit; an operand at byte offset x is the
+        // base plus x/16
+        const uint64_t ad = smem_desc_sw128(a0, 16, a_sbo);
+        const uint64_t bdd = smem_desc_sw128(b0, 16, 1024);
         for (int j = 0; j < kgroup; ++j) {
+          const uint64_t aj = ad + (uint64_t)((j * a_jstride) >> 4);
+          const uint64_t bj = bdd + (uint64_t)((j * n_tile * kProjKBlock * 2) >> 4);
 #pragma unroll
-          for (int k = 0; k < kProjKBlock / 16; ++k) {  // 32 bytes of k per step inside the 128-byte rows
-            const uint64_t a = smem_desc_sw128(a0 + j * a_jstride + k * 32, 16, a_sbo);
-            const uint64_t bd = smem_desc_sw128(b0 + j * n_tile * kProjKBlock * 2 + k * 32, 16, 1024);
-            mma_ss(tmem + acc * acc_cols, a, bd, idesc, (first && j == 0 && k == 0) ? 0u : 1u);
-          }
+          for (int k = 0; k < kProjKBlock / 16; ++k)  // 32 bytes of k per step inside the 128-byte rows
+            mma_ss(tmem + acc * acc_cols, aj + (uint64_t)(k * 2), bj + (uint64_t)(k * 2), idesc,
+                   (first && j == 0 && k == 0) ? 0u : 1u);
         }
         mma_commit(empty(st));
         if (last) {
