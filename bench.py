@@ -625,12 +625,13 @@ def e2e_measurement(args, dec, sets, w, device, stream, world, n_streams=3):
     names = ("q_nope", "q_pe", "end_pos", "topk_idx")
     # each set's inputs in one pinned buffer laid out like the staging area:
     # the entry point uploads them in one copy
-    hins = []
+    hins, hbufs = [], []
     for s_ in sets:
-        _, views = binding.host_input_buffer(B, K, S_max)
+        hbuf, views = binding.host_input_buffer(B, K, S_max)
         for k in names:
             views[k].copy_(s_["host"][k])
         hins.append(views)
+        hbufs.append(hbuf)
     houts = [torch.empty((B, 128, 128), dtype=torch.bfloat16).pin_memory() for _ in range(n_streams)]
     hws = [torch.empty(api.host_workspace_size(B, K, S_max), dtype=torch.uint8, device=device)
            for _ in range(n_streams)]
@@ -669,11 +670,60 @@ def e2e_measurement(args, dec, sets, w, device, stream, world, n_streams=3):
     repeats = max(1, min(10000, math.ceil(500.0 / max(probe, 1e-3))))
     wins = [max_over_ranks(window(args.steps), world, device) for _ in range(repeats)]
     e_ms = statistics.median(wins)
+    ceiling = copy_ceiling(args, hbufs, houts, streams, world, device)
+    ceiling["frac"] = whole_job_rate(B, world, args.steps, e_ms) / ceiling["value"]
     return {"value": whole_job_rate(B, world, args.steps, e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "windows": repeats,
+            "d2h_bytes_per_step": d2h, "windows": repeats, "copy_bound": ceiling,
             "how": f"per step one mla_sparse_decode_host call (the step's inputs uploaded from one pinned host "
                    f"buffer in one copy, decode, result read back to pinned memory, all on the call's stream); "
                    f"steps rotate over {n_streams} streams; median of {repeats} windows of {args.steps} steps"}
+
+
+def copy_ceiling(args, hbufs, houts, streams, world, device):
+    """What the copies allow: the step's packed input upload (pinned host ->
+    device, one copy) and its output read-back (device -> pinned host), timed
+    back to back with no kernels, each direction alone and both at once on two
+    streams.  The upload is the larger of the two, so a step can take no less
+    than the upload alone: `value` is that rate in queries/s, the ceiling of
+    the end-to-end figure whatever the kernels do (frac = end to end / it)."""
+    n = max(args.steps, 50)
+    up_bytes, down_bytes = hbufs[0].numel(), houts[0].numel() * houts[0].element_size()
+    dev_in = [torch.empty(up_bytes, dtype=torch.uint8, device=device) for _ in range(2)]
+    dev_out = torch.empty(down_bytes, dtype=torch.uint8, device=device)
+    outs = [o.view(torch.uint8).view(-1) for o in houts]
+    s_up, s_down = streams[0], streams[1]
+
+    def run(up: bool, down: bool) -> float:
+        ev = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in ("u", "d")}
+        start = torch.cuda.Event()
+        start.record(s_up)
+        s_down.wait_event(start)
+        ev["u"][0].record(s_up)
+        ev["d"][0].record(s_down)
+        for i in range(n):
+            if up:
+                with torch.cuda.stream(s_up):
+                    dev_in[i % 2].copy_(hbufs[i % len(hbufs)], non_blocking=True)
+            if down:
+                with torch.cuda.stream(s_down):
+                    outs[i % len(outs)].copy_(dev_out, non_blocking=True)
+        ev["u"][1].record(s_up)
+        ev["d"][1].record(s_down)
+        torch.cuda.synchronize()
+        t = max(ev["u"][0].elapsed_time(ev["u"][1]) if up else 0.0, ev["d"][0].elapsed_time(ev["d"][1]) if down else 0.0)
+        return max_over_ranks(t, world, device) / n
+
+    for _ in range(3):
+        run(True, True)
+    up_ms = statistics.median(run(True, False) for _ in range(5))
+    down_ms = statistics.median(run(False, True) for _ in range(5))
+    both_ms = statistics.median(run(True, True) for _ in range(5))
+    B = houts[0].shape[0]
+    return {"value": whole_job_rate(B, world, 1, up_ms), "unit": UNIT, "upload_ms_per_step": up_ms,
+            "readback_ms_per_step": down_ms, "both_ms_per_step": both_ms,
+            "h2d_gbs": up_bytes / up_ms / 1e6, "d2h_gbs": down_bytes / down_ms / 1e6,
+            "how": f"{n} copies back to back, no kernels: the {up_bytes}-byte packed upload alone (value), the "
+                   f"{down_bytes}-byte read-back alone, and both at once on two streams (both_ms_per_step)"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
