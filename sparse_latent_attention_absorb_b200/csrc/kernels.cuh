@@ -200,11 +200,15 @@ absorb_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 //
 // Warp roles (448 threads): warps 0-3 softmax group 0 (even tiles), warps
 // 4-7 softmax group 1 (odd tiles), warp w covering TMEM lanes 32(w%4)..;
-// warp 8 TMEM allocation, the query's tensor-map loads and QK issue; warp 9
-// PV issue; warps 10-13 gather (sixteen rows of every tile each).  QK and PV
-// are issued by different threads: their MMAs interleave in the tensor pipe,
-// and a commit (which tracks the issuing thread's MMAs only) signals PV
-// completion without waiting for a QK queued ahead of it.
+// warp 10 TMEM allocation, the query's tensor-map loads and QK issue; warp 9
+// PV issue; warps 8, 11, 12 and 13 gather (sixteen rows of every tile each).
+// QK and PV are issued by different threads: their MMAs interleave in the
+// tensor pipe, and a commit (which tracks the issuing thread's MMAs only)
+// signals PV completion without waiting for a QK queued ahead of it.  Warp w
+// runs on SM sub-partition w % 4, beside the two softmax warps of TMEM lane
+// quarter w % 4.  The QK thread sits on sub-partition 2, beside no gather or
+// PV warp: next to the quarter-0 softmax warps (as warp 8) it made them the
+// last of their group to finish nearly every tile.
 // =============================================================================
 constexpr int kNt = 64;                            // positions per tile
 constexpr int kStages = 4;                         // gathered tile ring
@@ -225,10 +229,13 @@ constexpr int kOffRed = kOffMslot + kMslotBytes;
 constexpr int kOffBar = kOffRed + kRedBytes;
 constexpr int kAttendSmemBytes = kOffBar + kBarBytes + kSmemAlignPad;
 constexpr int kSoftmaxWarps = 8;                   // two groups of four
-constexpr int kMmaWarp = 8;     // TMEM allocation, QK issue
-constexpr int kPvWarp = 9;      // PV issue
-constexpr int kGatherWarp0 = 10;
+constexpr int kMmaWarp = 10;    // TMEM allocation, QK issue (sub-partition 2)
+constexpr int kPvWarp = 9;      // PV issue (sub-partition 1)
 constexpr int kGatherWarps = 4;  // gather warp g fills rows 16g..16g+15 of every tile
+// Gather warp index g of warp 8, 11, 12, 13 (sub-partitions 0, 3, 0, 1), or -1.
+__device__ __forceinline__ int gather_index(int warp) {
+  return warp == 8 ? 0 : (warp >= 11 && warp <= 13 ? warp - 10 : -1);
+}
 // PV(j) is issued after QK(j + kPvLag).  QK(j + kPvLag) needs the stage of
 // tile j + kPvLag - kStages, freed by that tile's PV: it must come before
 // PV(j), or PV(j) would wait for itself.  A lag of 3 keeps PV out of the QK
@@ -238,7 +245,7 @@ constexpr int kPvLag = 2;
 static_assert(kPvLag < kStages, "PV may not wait for a QK that needs its own stage");
 // 14 warps: at most 128 registers a thread (the warps spread over the four
 // SM sub-partitions, 16K registers each, two of which hold four warps).
-constexpr int kAttendThreads = 32 * (kGatherWarp0 + kGatherWarps);  // 448
+constexpr int kAttendThreads = 32 * (kSoftmaxWarps + 2 + kGatherWarps);  // 448: warps 0..13
 // TMEM columns
 constexpr uint32_t kColS = 0;     // the score buffer (f32)
 constexpr uint32_t kColP = 64;    // P buffer of group g at kColP + 32g (bf16 pairs)
@@ -257,7 +264,7 @@ static_assert(kColS + kNt <= kColP && kColP + kNt <= kColQ && kColQ + 128 <= kCo
 // phases two apart).  For the same reason a warp never arrives twice on one
 // phase of kv_full.
 static_assert(kGatherWarps * 16 == kNt, "sixteen rows of a tile per gather warp");
-static_assert(kMmaWarp == kSoftmaxWarps && kPvWarp == kMmaWarp + 1 && kGatherWarp0 == kPvWarp + 1, "warp roles");
+static_assert(kAttendThreads == 14 * 32 && kMmaWarp == 10 && kPvWarp == 9, "warp roles: 0-7 softmax, 9 PV, 10 QK, the rest gather");
 
 struct AttendBars {
   uint64_t q_tma;               // the query boxes (TMA, transaction bytes) landed
@@ -456,7 +463,7 @@ sparse_attend_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_c
   if (tid == 0) MLA_CLUSTER_STAMP(kCeStart);
 #endif
 
-  if (warp >= kGatherWarp0) {
+  if (gather_index(warp) >= 0) {
     // ------------------------------------------------------------ gather
     // All four gather warps fill every tile: warp g copies rows
     // [16g, 16g + 16) of it (latent: one row per instruction, 32 lanes x 16
@@ -465,7 +472,7 @@ sparse_attend_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_c
     // A tile is published (kv_full, one arrival per warp) once every warp's
     // copies have landed.  Each warp visits the stages in tile order, so its
     // successive waits on one stage's kv_empty are exactly one phase apart.
-    const int g = warp - kGatherWarp0;
+    const int g = gather_index(warp);
     const int row0 = 16 * g;
     const __nv_bfloat16* kv_row0 = kv_cache + (size_t)slot * S_max * kDl + rank * 256;
     const __nv_bfloat16* pe_row0 = pe_cache + (size_t)slot * S_max * kDr + rank * 32;
